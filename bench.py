@@ -1,0 +1,421 @@
+"""Benchmark of the sparse MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the whole layer (router, gate/top-k or RRE, slot
+assignment, dispatch, expert FFN, combine) over one batch of T synthetic
+tokens.  The device-timed loop calls the layer stage by stage through the C
+ABI with CUDA events between the stages (same kernels, same stream as
+``moe_layer_forward``), so the step time and each stage's time come from one
+run.  ``e2e`` times ``moe_layer_forward`` itself with the batch copied from
+pinned host memory and the output copied back inside the timed region.
+
+Multi-GPU (torchrun): every rank runs its own batch with replicated experts
+(weak scaling, no collective on the data path); timing is the max over ranks.
+``--impl reference`` times the CPU oracle instead, on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="switch_base", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline object)
+# ---------------------------------------------------------------------------
+
+def oracle_step_fn(w, T_s):
+    """A closure running the oracle's whole layer on the first T_s tokens of the workload."""
+    import oracle
+    ws = w.scaled(T=T_s)
+    inp = synth.layer_inputs(ws)
+    C = oracle.capacity(ws.T, ws.E, ws.capacity_factor)
+    nth = os.cpu_count() or 1
+
+    def step():
+        oracle.layer_forward(inp["x"], inp["W1"], inp["W2"], E=ws.E, k=ws.k, C=C, Wr=inp["Wr"],
+                             bias=inp["bias"], domain=inp["domain"], G=ws.num_groups, seed=ws.seed,
+                             nthreads=nth)
+    return step, nth
+
+
+def size_oracle_sample(w, seconds):
+    """Pick a token count whose oracle step takes about `seconds`."""
+    T_s = 32
+    step, _ = oracle_step_fn(w, T_s)
+    t0 = time.perf_counter()
+    step()
+    dt = max(1e-3, time.perf_counter() - t0)
+    return int(max(32, min(w.T, T_s * seconds / dt)))
+
+
+def cpu_baseline(w, seconds):
+    T_s = size_oracle_sample(w, seconds / 2)
+    step, nth = oracle_step_fn(w, T_s)
+    t0 = time.perf_counter()
+    step()
+    dt = time.perf_counter() - t0
+    return {"value": T_s / dt, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+            "sample": f"whole layer on the first {T_s} of {w.T} tokens (capacity from eq. 3 at "
+                      f"T={T_s}), fp64 CPU oracle, {nth} threads, one timed pass of {dt:.2f} s"}
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    T_s = size_oracle_sample(w, 1.0)
+    step, nth = oracle_step_fn(w, T_s)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = T_s * args.steps / dt
+    out = {"impl": "reference", "metric": "MoE-layer tokens/sec", "value": value,
+           "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff,
+                      "E": w.E, "k": w.k, "capacity_factor": w.capacity_factor,
+                      "routing": w.mode, "tokens_per_step_sampled": T_s},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+                            "sample": f"whole layer on the first {T_s} of {w.T} tokens per step"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the B200 arm
+# ---------------------------------------------------------------------------
+
+def run_b200(args, w, world, rank, local):
+    import sparse_mixture_experts_fwd_b200 as moe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    es = 2 if w.dtype == "bf16" else 4
+    C = moe.capacity(w.T, w.E, w.capacity_factor)
+    cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, C, dtype=w.torch_dtype, mode=w.mode,
+                          num_groups=w.num_groups, seed=w.seed)
+    inp = synth.layer_inputs(w, x_seed_offset=rank)
+    W1, W2 = inp["W1"].to(dev), inp["W2"].to(dev)
+    Wr = None if inp["Wr"] is None else inp["Wr"].to(dev)
+    bias = None if inp["bias"] is None else inp["bias"].to(dev)
+    x_bytes = w.T * w.d_model * es
+    n_rot = max(2, -(-2 * L2_BYTES // x_bytes))  # rotate batches: > 2x L2 of distinct x
+    xs = [inp["x"].to(dev)]
+    doms = [None if inp["domain"] is None else inp["domain"].to(dev)]
+    gen_extra = synth.layer_inputs
+    for r in range(1, n_rot):
+        extra = gen_extra(w, weights=False, x_seed_offset=rank + 1000 * r)
+        xs.append(extra["x"].to(dev))
+        doms.append(None if extra["domain"] is None else extra["domain"].to(dev))
+    ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    v = moe.workspace_views(cfg, ws)
+    y = torch.empty(w.T, w.d_model, dtype=w.torch_dtype, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    asg = {k: v[k] for k in ("expert_idx", "gate", "slot", "kept", "tok_of_row", "arrivals",
+                             "kept_cnt", "n_dropped")}
+    scratch = ws[moe.workspace_layout(cfg).scratch:]
+    logits = v.get("logits")
+
+    stage_names = ["router", "route_assign", "dispatch", "expert_ffn", "combine"]
+
+    def step(i, evs=None):
+        x = xs[i % n_rot]
+        dom = doms[i % n_rot]
+        if evs:
+            evs[0].record(stream)
+        if w.mode == "topk":
+            moe.router(cfg, x, Wr, bias, logits=logits, status=status, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        moe.topk_assign(cfg, logits=logits, domain_id=dom, out=asg, workspace=scratch,
+                        status=status, stream=stream)
+        if evs:
+            evs[2].record(stream)
+        moe.dispatch(cfg, x, asg["expert_idx"], asg["slot"], asg["kept"], xe=v["xe"], stream=stream)
+        if evs:
+            evs[3].record(stream)
+        moe.expert_ffn(cfg, v["xe"], W1, W2, asg["kept_cnt"], H=v["H"], ye=v["ye"], status=status,
+                       stream=stream)
+        if evs:
+            evs[4].record(stream)
+        moe.combine(cfg, v["ye"], asg["expert_idx"], asg["gate"], asg["slot"], asg["kept"], y=y,
+                    stream=stream)
+        if evs:
+            evs[5].record(stream)
+
+    launches_per_step = (1 if w.mode == "topk" else 0) + 1 + 3 + 1 + 2 + 1
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                step(args.warmup + i, evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    total_ms = evs[0][0].elapsed_time(evs[-1][5])
+    stage_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
+                for j, n in enumerate(stage_names)}
+    total_ms_max = max_over_ranks(total_ms, world)
+
+    # routing statistics of the last step (same every step up to x)
+    kept_cnt = asg["kept_cnt"].cpu()
+    n_kept = int(kept_cnt.sum())
+    n_dropped = int(asg["n_dropped"].item())
+    tok_any = int((asg["kept"].cpu().sum(1) > 0).sum())
+
+    # algorithmic work of the dominant stage (expert FFN) and of dispatch + combine
+    ffn_bytes = 2 * w.E * w.d_model * w.d_ff * es + 2 * n_kept * w.d_model * es
+    ffn_flops = 4.0 * n_kept * w.d_model * w.d_ff
+    ffn_s = stage_ms["expert_ffn"] / 1e3
+    disp_bytes = (tok_any + n_kept) * w.d_model * es + 9 * w.T * w.k
+    comb_bytes = (n_kept + w.T) * w.d_model * es + 9 * w.T * w.k
+    dc_s = (stage_ms["dispatch"] + stage_ms["combine"]) / 1e3
+    intensity = ffn_flops / ffn_bytes
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity < ridge:
+        roof = {"bound": "hbm", "achieved": ffn_bytes / ffn_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": ffn_flops / ffn_s / 1e12,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "expert FFN: gemm_tc_kernel x2 (H = ReLU(xe W1^T), ye = H W2^T)"
+    roof["peak_source"] = peaks["source"]
+    roof["algorithmic_per_launch"] = (f"{ffn_bytes / 1e9:.4f} GB" if roof["bound"] == "hbm"
+                                      else f"{ffn_flops / 1e12:.4f} TFLOP")
+
+    # ---- e2e through moe_layer_forward with host buffers ----
+    xh = [torch.empty_like(xs[r], device="cpu").pin_memory() for r in range(min(n_rot, 4))]
+    for r in range(len(xh)):
+        xh[r].copy_(xs[r].cpu())
+    dh = None
+    if w.mode == "rre":
+        dh = [doms[r].cpu().pin_memory() for r in range(len(xh))]
+    yh = torch.empty(w.T, w.d_model, dtype=w.torch_dtype).pin_memory()
+    xd = torch.empty_like(xs[0])
+    dd = None if dh is None else torch.empty_like(doms[0])
+    h2d = x_bytes + (w.T * 4 if dh is not None else 0)
+    d2h = x_bytes
+
+    def e2e_step(i):
+        xd.copy_(xh[i % len(xh)], non_blocking=True)
+        if dd is not None:
+            dd.copy_(dh[i % len(dh)], non_blocking=True)
+        moe.layer_forward(cfg, xd, W1, W2, Wr=Wr, bias=bias, domain_id=dd, y=y, workspace=ws,
+                          status=status, stream=stream)
+        yh.copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    tokens_all = sum_over_ranks(float(w.T * args.steps), world)
+    value = tokens_all / (total_ms_max / 1e3)
+    e2e_value = tokens_all / (e2e_ms / 1e3)
+
+    if rank != 0:
+        return
+    clocks = clk.summary()
+    out = {
+        "metric": "MoE-layer tokens/sec (1 B200); expert-FFN TFLOP/s; dispatch+combine GB/s",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E,
+                   "k": w.k, "capacity_factor": w.capacity_factor, "capacity": C,
+                   "routing": w.mode, "tokens_per_rank_per_step": w.T,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"x rotated over {n_rot} batches ({n_rot * x_bytes / 2**20:.0f} MiB) and "
+                         f"expert weights {2 * w.E * w.d_model * w.d_ff * es / 2**30:.2f} GiB, "
+                         "both larger than the 126 MB L2"},
+        "roofline": roof,
+        "stages_ms": {k: round(v_, 5) for k, v_ in stage_ms.items()},
+        "expert_ffn_tflops": ffn_flops / ffn_s / 1e12,
+        "dispatch_combine_gbs": (disp_bytes + comb_bytes) / dc_s / 1e9,
+        "routing": {"n_kept": n_kept, "n_dropped": n_dropped,
+                    "drop_rate": n_dropped / (w.T * w.k)},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "api": "moe_layer_forward"},
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    world, rank, local = (1, 0, 0)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_b200(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * moe_b200.h — C ABI of the sparse Mixture-of-Experts layer forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (page "Switch Transformers: Scaling to Trillion Parameter Models
+ * with Simple and Efficient Sparsity", study notes, sec. 2.1-2.2):
+ *   router      h(x) = W_r x                                  (sec. 2.1)
+ *   gate        p_i(x) = exp(h_i) / sum_j exp(h_j)            (sec. 2.1, eq. 1)
+ *   top-k set   T = indices of the k largest gates            (sec. 2.1; k = 1
+ *               Switch, k = 2 X-MoE per "[Paper review] TorchScale",
+ *               proposed method)
+ *   capacity    C = (tokens / experts) x capacity_factor      (sec. 2.2, eq. 3)
+ *               overflowing tokens are dropped: the layer adds 0 for them
+ *   experts     E_i(x) = ReLU(x W1_i^T) W2_i^T
+ *   combine     y = sum_{i in T} p_i(x) E_i(x)                (sec. 2.1, eq. 2)
+ * plus Random Routed Experts ("[Paper review] PanGu-Sigma", proposed method)
+ * and the SparseClip norm ("[Paper review] TorchScale", proposed method).
+ *
+ * Conventions for every entry point:
+ *   * All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains device memory.  Scratch comes
+ *     from a caller-provided workspace of the size the matching *_size query
+ *     returns.  Host-side arrays are marked "host".
+ *   * Tensors are dense, row-major (C order), 16-byte aligned.  Activations
+ *     and weights are bf16 (dtype MOE_DTYPE_BF16) or fp32 (MOE_DTYPE_F32);
+ *     logits and gates are always fp32; indices int32; masks uint8.
+ *   * Work is enqueued asynchronously on `stream` (a cudaStream_t; 0 = the
+ *     legacy default stream) and the call returns at once.
+ *   * Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and returns a negative MOE_ERR_* code.
+ *     A failed launch returns MOE_ERR_CUDA; moe_last_error() describes it.
+ *   * Conditions seen on the device are OR-ed into the optional `status`
+ *     word (device int32, nullable; enum moe_status_bits).  The caller
+ *     zeroes `status` before the call and reads it after synchronising.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+#define MOE_ABI_VERSION 1
+
+enum moe_error {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARGUMENT = -1, /* null pointer, bad size, bad enum value   */
+  MOE_ERR_UNSUPPORTED = -2,      /* valid MoE, but outside this build's range */
+  MOE_ERR_ALIGNMENT = -3,        /* pointer not 16-byte aligned               */
+  MOE_ERR_WORKSPACE = -4,        /* workspace missing or too small            */
+  MOE_ERR_CUDA = -5              /* a CUDA runtime / driver call failed       */
+};
+
+enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 };
+enum moe_route_mode { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RRE = 1 };
+enum moe_status_bits {
+  MOE_STATUS_TIMEOUT = 1,   /* a pipeline wait gave up after 1 s; outputs invalid     */
+  MOE_STATUS_BAD_DOMAIN = 2 /* an RRE domain id was outside 0..G-1 (routed as 0)       */
+};
+
+/* One MoE layer.  48 bytes, no padding. */
+typedef struct moe_config {
+  int64_t T;          /* tokens in the batch (>= 0)                                    */
+  int32_t d_model;    /* token width d                                                 */
+  int32_t d_ff;       /* expert hidden width f                                         */
+  int32_t E;          /* experts, 1..256                                               */
+  int32_t k;          /* experts per token: 1 or 2 (RRE: 1)                            */
+  int32_t capacity;   /* C, tokens per expert (>= 0); see moe_capacity                 */
+  int32_t mode;       /* enum moe_route_mode                                           */
+  int32_t num_groups; /* RRE: G domain groups, E % G == 0; ignored for TOPK            */
+  int32_t dtype;      /* enum moe_dtype of x, W_r, W1, W2, xe, H, ye, y                */
+  uint64_t seed;      /* RRE: seed of the splitmix64 routing hash; ignored for TOPK    */
+} moe_config;
+
+/* Workspace layout used by moe_layer_forward: byte offsets from the
+ * workspace base (each 256-byte aligned) and the total size.  After a call
+ * the caller may read any of these intermediate tensors. */
+typedef struct moe_workspace_map {
+  size_t logits;     /* [T, E] fp32 (TOPK only)                 */
+  size_t expert_idx; /* [T, k] int32                            */
+  size_t gate;       /* [T, k] fp32                             */
+  size_t slot;       /* [T, k] int32                            */
+  size_t kept;       /* [T, k] uint8                            */
+  size_t tok_of_row; /* [E, C] int32, -1 where the slot is free */
+  size_t arrivals;   /* [E] int32                               */
+  size_t kept_cnt;   /* [E] int32                               */
+  size_t n_dropped;  /* [1] int32                               */
+  size_t scratch;    /* assignment scratch (moe_assign_workspace_size bytes) */
+  size_t xe;         /* [E, C, d] activations                   */
+  size_t H;          /* [E, C, f] activations                   */
+  size_t ye;         /* [E, C, d] activations                   */
+  size_t total;
+} moe_workspace_map;
+
+/* ---- host-only queries (no CUDA call) --------------------------------- */
+
+int32_t moe_abi_version(void);
+/* sizeof(moe_config) and sizeof(moe_workspace_map) as compiled, for binders. */
+size_t moe_config_size(void);
+size_t moe_workspace_map_size(void);
+/* Static text for an enum moe_error value. */
+const char* moe_error_string(int32_t code);
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char* moe_last_error(void);
+
+/* Eq. (3) of the Switch notes, sec. 2.2: floor(T / E * capacity_factor).
+ * Returns -1 if E < 1, T < 0 or capacity_factor < 0. */
+int32_t moe_capacity(int64_t T, int32_t E, double capacity_factor);
+
+/* MOE_OK if `cfg` is a layer this build runs, else the error code. */
+int32_t moe_config_check(const moe_config* cfg);
+
+/* Bytes of scratch moe_topk_assign needs (0 if cfg is invalid). */
+size_t moe_assign_workspace_size(const moe_config* cfg);
+
+/* Layout (and total size) of the moe_layer_forward workspace. */
+int32_t moe_workspace_layout(const moe_config* cfg, moe_workspace_map* out);
+size_t moe_workspace_size(const moe_config* cfg); /* 0 if cfg is invalid */
+
+/* Bytes of scratch sparseclip_norm needs for this many tensors. */
+size_t sparseclip_workspace_size(int32_t n_dense, int32_t n_sparse);
+
+/* ---- the layer, step by step ------------------------------------------ */
+
+/* Router logits (Switch notes sec. 2.1; fp32 router per sec. 2.4):
+ *   logits[t, e] = sum_c x[t, c] * Wr[e, c] (+ bias[e])
+ * x [T, d] and Wr [E, d] in cfg->dtype; bias [E] fp32, nullable; logits
+ * [T, E] fp32.  bf16 inputs: exact products, fp32 accumulation on the
+ * tensor cores (requires E % 16 == 0).  fp32 inputs: fp32 FMA chain. */
+int32_t moe_router(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
+                   float* logits, int32_t* status, moe_stream_t stream);
+
+/* Gate, expert choice and capacity-bounded slot assignment.
+ * TOPK (Switch notes sec. 2.1 eq. 1, sec. 2.2 eq. 3): from logits [T, E]
+ *   pick the k largest (ties -> lower expert index), gate[t, j] = the
+ *   softmax probability of that expert over all E (no renormalisation).
+ * RRE ("[Paper review] PanGu-Sigma", proposed method): from domain_id [T]
+ *   (values 0..G-1) pick expert domain*(E/G) + splitmix64(seed, t) mod
+ *   (E/G), gate 1.  logits unused (may be null).
+ * Then, in token order (token t's choices before token t+1's), slot[t, j] =
+ *   number of earlier choices of the same expert; kept[t, j] = slot < C;
+ *   tok_of_row[e*C + s] = token in slot s of expert e, -1 if none;
+ *   arrivals[e] = choices of e; kept_cnt[e] = min(arrivals[e], C);
+ *   n_dropped[0] = sum_e max(0, arrivals[e] - C).
+ * Outputs: expert_idx, slot [T, k] int32; gate [T, k] fp32; kept [T, k]
+ * uint8; tok_of_row [E*C] int32; arrivals, kept_cnt [E] int32; n_dropped
+ * [1] int32.  workspace: moe_assign_workspace_size(cfg) bytes. */
+int32_t moe_topk_assign(const moe_config* cfg, const float* logits, const int32_t* domain_id,
+                        int32_t* expert_idx, float* gate, int32_t* slot, uint8_t* kept,
+                        int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
+                        int32_t* n_dropped, void* workspace, size_t workspace_bytes,
+                        int32_t* status, moe_stream_t stream);
+
+/* Dispatch (the permutation the Switch router's dispatch tensor encodes,
+ * sec. 2.4): xe[e, s, :] = x[t, :] for every kept choice (t, j) with
+ * e = expert_idx[t, j], s = slot[t, j].  Rows of xe that no token fills are
+ * left untouched.  x [T, d], xe [E, C, d] in cfg->dtype. */
+int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert_idx,
+                     const int32_t* slot, const uint8_t* kept, void* xe, moe_stream_t stream);
+
+/* Expert FFNs as one grouped computation over the kept rows:
+ *   H[e, r, :]  = round(ReLU(xe[e, r, :] . W1[e]^T))   W1 [E, f, d]
+ *   ye[e, r, :] = round(H[e, r, :] . W2[e]^T)          W2 [E, d, f]
+ * for r < kept_cnt[e] (device int32 [E], values in 0..C).  xe, ye
+ * [E, C, d] and H [E, C, f] (caller-provided scratch) in cfg->dtype; other
+ * rows of H and ye are left untouched.  bf16: tcgen05 tensor cores with
+ * fp32 accumulation; fp32: FMA. */
+int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
+                       const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
+                       moe_stream_t stream);
+
+/* Combine (Switch notes sec. 2.1, eq. 2; drop rule sec. 2.2):
+ *   y[t, :] = sum over kept j of gate[t, j] * ye[expert_idx[t, j], slot[t, j], :]
+ * accumulated in fp32 and rounded once; 0 for a token with no kept choice.
+ * y [T, d] in cfg->dtype. */
+int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert_idx,
+                    const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
+                    moe_stream_t stream);
+
+/* The whole layer: router (TOPK) -> gate/top-k or RRE -> slot assignment ->
+ * dispatch -> expert FFN -> combine, all on `stream`.  Wr (+ bias) for TOPK,
+ * domain_id for RRE (the other may be null).  y [T, d] in cfg->dtype.
+ * workspace: moe_workspace_size(cfg) bytes laid out as moe_workspace_layout
+ * describes; it holds every intermediate after the call. */
+int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
+                          const int32_t* domain_id, const void* W1, const void* W2, void* y,
+                          void* workspace, size_t workspace_bytes, int32_t* status,
+                          moe_stream_t stream);
+
+/* SparseClip global gradient norm ("[Paper review] TorchScale", proposed
+ * method): ||g||_2 = ||(g_d, kappa g_s)||_2 with kappa = 1/sqrt(num_experts),
+ *   out[0] = sqrt(Sd + Ss / num_experts), out[1] = Sd, out[2] = Ss,
+ *   Sd = sum of squares over the dense tensors, Ss over the expert tensors.
+ * dense / sparse: host arrays of device fp32 pointers with host arrays of
+ * element counts; out: device double[3].  Squares are summed in fp32 over
+ * groups of 4 elements and in fp64 above that, in a fixed order, so the
+ * result is the same on every run on the same GPU model.  n_dense + n_sparse
+ * <= 4096.  workspace: sparseclip_workspace_size(n_dense, n_sparse) bytes. */
+int32_t sparseclip_norm(const float* const* dense, const int64_t* dense_len, int32_t n_dense,
+                        const float* const* sparse, const int64_t* sparse_len, int32_t n_sparse,
+                        int32_t num_experts, double* out, void* workspace, size_t workspace_bytes,
+                        moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

@@ -51,6 +51,7 @@ def _load():
         "oracle_expert_row": ([i32, i32, i32, vp, vp, vp, vp, vp], None),
         "oracle_expert_ffn": ([i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32], None),
         "oracle_combine": ([i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], None),
+        "oracle_token_forward": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp], None),
         "oracle_layer_forward": ([i64, i32, i32, i32, i32, i32, i32, i32, i32, u64] + [vp] * 19
                                  + [i32], None),
         "oracle_sparseclip_norm": ([vp, vp, i32, vp, vp, i32, i32], dbl),
@@ -166,6 +167,17 @@ def combine(ye, expert_idx, gate, slot, kept, T):
     y = torch.empty(T, d, dtype=ye.dtype)
     _load().oracle_combine(T, d, k, C, _dt(ye), _p(ye), _p(expert_idx), _p(gate), _p(slot),
                            _p(kept), _p(y))
+    return y
+
+
+def token_forward(x_row, W1, W2, expert_idx_row, gate_row, kept_row):
+    """Layer output of one token (eq. (2) for a single x) from full W1 [E,f,d], W2 [E,d,f]."""
+    E, f, d = W1.shape
+    k = expert_idx_row.numel()
+    y = torch.empty(d, dtype=x_row.dtype)
+    _load().oracle_token_forward(d, f, k, _dt(x_row), _p(x_row.contiguous()), _p(W1), _p(W2),
+                                 _p(expert_idx_row.contiguous()), _p(gate_row.contiguous()),
+                                 _p(kept_row.contiguous()), _p(y))
     return y
 
 

@@ -295,6 +295,27 @@ void oracle_combine(int64_t T, int32_t d, int32_t k, int32_t C, int32_t dtype, c
     }
 }
 
+// One token's layer output (eq. (2) for a single x): y = sum over its kept
+// choices j of gate_j * E_{e_j}(x), each expert output rounded as in
+// oracle_expert_row, the sum in double and rounded once.  W1 [E, f, d] and
+// W2 [E, d, f] are the full weight tensors.
+void oracle_token_forward(int32_t d, int32_t f, int32_t k, int32_t dtype, const void* x_row,
+                          const void* W1, const void* W2, const int32_t* expert_idx_row,
+                          const float* gate_row, const uint8_t* kept_row, void* y_row) {
+  const size_t es = dtype == DT_BF16 ? 2 : 4;
+  std::vector<double> acc(d, 0.0);
+  std::vector<uint32_t> out(d);  // room for d fp32 or bf16 values
+  for (int32_t j = 0; j < k; ++j) {
+    if (!kept_row[j]) continue;
+    const int64_t e = expert_idx_row[j];
+    oracle_expert_row(d, f, dtype, x_row, static_cast<const char*>(W1) + e * f * d * es,
+                      static_cast<const char*>(W2) + e * d * f * es, out.data(), nullptr);
+    for (int32_t c = 0; c < d; ++c)
+      acc[c] += static_cast<double>(gate_row[j]) * load(out.data(), c, dtype);
+  }
+  for (int32_t c = 0; c < d; ++c) store(y_row, c, dtype, acc[c]);
+}
+
 // The whole layer, step by step, in the pages' order.  mode 0: softmax
 // gate + top-k (Wr, bias used); mode 1: RRE (domain, seed, G used; k = 1).
 // Buffers the caller may inspect: logits [T,E] (mode 0), expert_idx/gate/

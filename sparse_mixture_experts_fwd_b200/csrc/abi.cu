@@ -1,0 +1,331 @@
+// C ABI entry points: argument validation, workspace layout and the layer
+// forward sequence.  Every device-side step is one of the library's kernels.
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+#include <string>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+thread_local std::string g_last_error;
+}
+
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
+const char* last_error_cstr() { return g_last_error.c_str(); }
+
+int32_t fail(int32_t code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+int32_t check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return MOE_OK;
+  return fail(MOE_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+constexpr int64_t kI32Max = 2147483647;
+
+int32_t check_cfg(const moe_config* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARGUMENT, "config is null");
+  if (c->T < 0 || c->T > kI32Max) return fail(MOE_ERR_INVALID_ARGUMENT, "T out of range");
+  if (c->E < 1) return fail(MOE_ERR_INVALID_ARGUMENT, "E < 1");
+  if (c->E > 256) return fail(MOE_ERR_UNSUPPORTED, "E > 256");
+  if (c->k != 1 && c->k != 2) return fail(MOE_ERR_UNSUPPORTED, "k must be 1 or 2");
+  if (c->k > c->E) return fail(MOE_ERR_INVALID_ARGUMENT, "k > E");
+  if (c->capacity < 0) return fail(MOE_ERR_INVALID_ARGUMENT, "capacity < 0");
+  if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_F32)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "unknown dtype");
+  if (c->mode != MOE_ROUTE_TOPK && c->mode != MOE_ROUTE_RRE)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "unknown routing mode");
+  if (c->mode == MOE_ROUTE_RRE) {
+    if (c->k != 1) return fail(MOE_ERR_INVALID_ARGUMENT, "RRE routes each token to one expert (k=1)");
+    if (c->num_groups < 1 || c->E % c->num_groups != 0)
+      return fail(MOE_ERR_INVALID_ARGUMENT, "RRE needs num_groups >= 1 dividing E");
+  }
+  if (c->d_model < 1 || c->d_ff < 1) return fail(MOE_ERR_INVALID_ARGUMENT, "d_model/d_ff < 1");
+  if (c->dtype == MOE_DTYPE_BF16) {
+    if (c->d_model % 64 || c->d_ff % 64)
+      return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d_model and d_ff multiples of 64");
+    if (c->mode == MOE_ROUTE_TOPK && c->E % 16)
+      return fail(MOE_ERR_UNSUPPORTED, "bf16 router needs E multiple of 16");
+  } else {
+    if (c->d_model % 4 || c->d_ff % 4)
+      return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d_model and d_ff multiples of 4");
+  }
+  const int64_t EC = int64_t(c->E) * c->capacity;
+  if (EC > kI32Max || int64_t(c->E) * c->d_ff > kI32Max || int64_t(c->E) * c->d_model > kI32Max)
+    return fail(MOE_ERR_UNSUPPORTED, "E*C, E*d_ff or E*d_model exceeds 2^31-1 rows");
+  return MOE_OK;
+}
+
+int32_t need_ptr(const void* p, const char* name, bool required = true) {
+  if (!p) {
+    if (!required) return MOE_OK;
+    return fail(MOE_ERR_INVALID_ARGUMENT, std::string(name) + " is null");
+  }
+  if (!aligned16(p)) return fail(MOE_ERR_ALIGNMENT, std::string(name) + " is not 16-byte aligned");
+  return MOE_OK;
+}
+
+// 4-byte-aligned pointers are enough for the per-token index/gate arrays.
+int32_t need_ptr4(const void* p, const char* name) {
+  if (!p) return fail(MOE_ERR_INVALID_ARGUMENT, std::string(name) + " is null");
+  if (reinterpret_cast<uintptr_t>(p) & 3u)
+    return fail(MOE_ERR_ALIGNMENT, std::string(name) + " is not 4-byte aligned");
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)              \
+  do {                             \
+    int32_t rc_ = (expr);          \
+    if (rc_ != MOE_OK) return rc_; \
+  } while (0)
+
+void layout(const moe_config& c, moe_workspace_map* m) {
+  const size_t es = elem_size(c.dtype);
+  const size_t T = static_cast<size_t>(c.T), k = static_cast<size_t>(c.k);
+  const size_t E = static_cast<size_t>(c.E), C = static_cast<size_t>(c.capacity);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  m->logits = take(c.mode == MOE_ROUTE_TOPK ? T * E * 4 : 0);
+  m->expert_idx = take(T * k * 4);
+  m->gate = take(T * k * 4);
+  m->slot = take(T * k * 4);
+  m->kept = take(T * k);
+  m->tok_of_row = take(E * C * 4);
+  m->arrivals = take(E * 4);
+  m->kept_cnt = take(E * 4);
+  m->n_dropped = take(4);
+  m->scratch = take(assign_scratch_bytes(c));
+  m->xe = take(E * C * static_cast<size_t>(c.d_model) * es);
+  m->H = take(E * C * static_cast<size_t>(c.d_ff) * es);
+  m->ye = take(E * C * static_cast<size_t>(c.d_model) * es);
+  m->total = off;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+size_t moe_config_size(void) { return sizeof(moe_config); }
+size_t moe_workspace_map_size(void) { return sizeof(moe_workspace_map); }
+
+const char* moe_error_string(int32_t code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_ALIGNMENT: return "pointer not aligned";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    default: return "unknown error";
+  }
+}
+
+const char* moe_last_error(void) { return last_error_cstr(); }
+
+int32_t moe_capacity(int64_t T, int32_t E, double capacity_factor) {
+  if (E < 1 || T < 0 || !(capacity_factor >= 0.0)) return -1;
+  const double c = std::floor(static_cast<double>(T) / E * capacity_factor);
+  return c > 2147483647.0 ? -1 : static_cast<int32_t>(c);
+}
+
+int32_t moe_config_check(const moe_config* cfg) {
+  set_last_error("");
+  return check_cfg(cfg);
+}
+
+size_t moe_assign_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return std::max<size_t>(256, assign_scratch_bytes(*cfg));
+}
+
+int32_t moe_workspace_layout(const moe_config* cfg, moe_workspace_map* out) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  if (!out) return fail(MOE_ERR_INVALID_ARGUMENT, "out is null");
+  layout(*cfg, out);
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  moe_workspace_map m;
+  layout(*cfg, &m);
+  return m.total;
+}
+
+int32_t moe_router(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
+                   float* logits, int32_t* status, moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  MOE_TRY(need_ptr(x, "x"));
+  MOE_TRY(need_ptr(Wr, "Wr"));
+  MOE_TRY(need_ptr(bias, "bias", false));
+  MOE_TRY(need_ptr(logits, "logits"));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MOE_DTYPE_BF16) {
+    if (cfg->E % 16) return fail(MOE_ERR_UNSUPPORTED, "bf16 router needs E multiple of 16");
+    return launch_router_tc(*cfg, x, Wr, bias, logits, status, s);
+  }
+  return launch_router_f32(*cfg, x, Wr, bias, logits, s);
+}
+
+int32_t moe_topk_assign(const moe_config* cfg, const float* logits, const int32_t* domain_id,
+                        int32_t* expert_idx, float* gate, int32_t* slot, uint8_t* kept,
+                        int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
+                        int32_t* n_dropped, void* workspace, size_t workspace_bytes,
+                        int32_t* status, moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  const bool any_tokens = cfg->T > 0;
+  if (any_tokens) {
+    if (cfg->mode == MOE_ROUTE_TOPK) MOE_TRY(need_ptr4(logits, "logits"));
+    else MOE_TRY(need_ptr4(domain_id, "domain_id"));
+    MOE_TRY(need_ptr4(expert_idx, "expert_idx"));
+    MOE_TRY(need_ptr4(gate, "gate"));
+    MOE_TRY(need_ptr4(slot, "slot"));
+    if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
+  }
+  if (int64_t(cfg->E) * cfg->capacity > 0) MOE_TRY(need_ptr4(tok_of_row, "tok_of_row"));
+  MOE_TRY(need_ptr4(arrivals, "arrivals"));
+  MOE_TRY(need_ptr4(kept_cnt, "kept_cnt"));
+  MOE_TRY(need_ptr4(n_dropped, "n_dropped"));
+  const size_t need = assign_scratch_bytes(*cfg);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(MOE_ERR_WORKSPACE, "moe_topk_assign: workspace needs " + std::to_string(need) + " bytes");
+  if (workspace) MOE_TRY(need_ptr(workspace, "workspace"));
+  return launch_route_assign(*cfg, logits, domain_id, expert_idx, gate, slot, kept, tok_of_row,
+                             arrivals, kept_cnt, n_dropped, workspace, status,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert_idx,
+                     const int32_t* slot, const uint8_t* kept, void* xe, moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->T == 0 || cfg->capacity == 0) return MOE_OK;
+  MOE_TRY(need_ptr(x, "x"));
+  MOE_TRY(need_ptr4(expert_idx, "expert_idx"));
+  MOE_TRY(need_ptr4(slot, "slot"));
+  if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
+  MOE_TRY(need_ptr(xe, "xe"));
+  return launch_dispatch(*cfg, x, expert_idx, slot, kept, xe, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
+                       const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
+                       moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->capacity == 0) return MOE_OK;
+  MOE_TRY(need_ptr(xe, "xe"));
+  MOE_TRY(need_ptr(W1, "W1"));
+  MOE_TRY(need_ptr(W2, "W2"));
+  MOE_TRY(need_ptr4(kept_cnt, "kept_cnt"));
+  MOE_TRY(need_ptr(H, "H"));
+  MOE_TRY(need_ptr(ye, "ye"));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MOE_DTYPE_BF16) return launch_ffn_tc(*cfg, xe, W1, W2, kept_cnt, H, ye, status, s);
+  return launch_ffn_f32(*cfg, xe, W1, W2, kept_cnt, H, ye, s);
+}
+
+int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert_idx,
+                    const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
+                    moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  if (cfg->capacity > 0) MOE_TRY(need_ptr(ye, "ye"));
+  MOE_TRY(need_ptr4(expert_idx, "expert_idx"));
+  MOE_TRY(need_ptr4(gate, "gate"));
+  MOE_TRY(need_ptr4(slot, "slot"));
+  if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
+  MOE_TRY(need_ptr(y, "y"));
+  return launch_combine(*cfg, ye, expert_idx, gate, slot, kept, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
+                          const int32_t* domain_id, const void* W1, const void* W2, void* y,
+                          void* workspace, size_t workspace_bytes, int32_t* status,
+                          moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  const moe_config& c = *cfg;
+  moe_workspace_map m;
+  layout(c, &m);
+  if (!workspace || workspace_bytes < m.total)
+    return fail(MOE_ERR_WORKSPACE, "moe_layer_forward: workspace needs " + std::to_string(m.total) + " bytes");
+  MOE_TRY(need_ptr(workspace, "workspace"));
+  if (c.T > 0) {
+    MOE_TRY(need_ptr(x, "x"));
+    MOE_TRY(need_ptr(y, "y"));
+    if (c.mode == MOE_ROUTE_TOPK) {
+      MOE_TRY(need_ptr(Wr, "Wr"));
+      MOE_TRY(need_ptr(bias, "bias", false));
+    } else {
+      MOE_TRY(need_ptr4(domain_id, "domain_id"));
+    }
+  }
+  if (c.capacity > 0) {
+    MOE_TRY(need_ptr(W1, "W1"));
+    MOE_TRY(need_ptr(W2, "W2"));
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* logits = reinterpret_cast<float*>(ws + m.logits);
+  int32_t* expert_idx = reinterpret_cast<int32_t*>(ws + m.expert_idx);
+  float* gate = reinterpret_cast<float*>(ws + m.gate);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + m.slot);
+  uint8_t* kept = reinterpret_cast<uint8_t*>(ws + m.kept);
+  int32_t* tok_of_row = reinterpret_cast<int32_t*>(ws + m.tok_of_row);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(ws + m.arrivals);
+  int32_t* kept_cnt = reinterpret_cast<int32_t*>(ws + m.kept_cnt);
+  int32_t* n_dropped = reinterpret_cast<int32_t*>(ws + m.n_dropped);
+  void* scratch = ws + m.scratch;
+  void* xe = ws + m.xe;
+  void* H = ws + m.H;
+  void* ye = ws + m.ye;
+
+  if (c.mode == MOE_ROUTE_TOPK && c.T > 0) {
+    if (c.dtype == MOE_DTYPE_BF16) MOE_TRY(launch_router_tc(c, x, Wr, bias, logits, status, s));
+    else MOE_TRY(launch_router_f32(c, x, Wr, bias, logits, s));
+  }
+  MOE_TRY(launch_route_assign(c, logits, domain_id, expert_idx, gate, slot, kept, tok_of_row,
+                              arrivals, kept_cnt, n_dropped, scratch, status, s));
+  MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, s));
+  if (c.dtype == MOE_DTYPE_BF16) MOE_TRY(launch_ffn_tc(c, xe, W1, W2, kept_cnt, H, ye, status, s));
+  else MOE_TRY(launch_ffn_f32(c, xe, W1, W2, kept_cnt, H, ye, s));
+  return launch_combine(c, ye, expert_idx, gate, slot, kept, y, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+// SparseClip global gradient norm ("[Paper review] TorchScale: Transformers
+// at Scale", proposed method):
+//   ||g||_2 = ||(g_d, kappa g_s)||_2 = sqrt(Sd + kappa^2 Ss),  kappa = 1/sqrt(E)
+// where Sd / Ss are the sums of squares of the dense / expert gradients.
+//
+// One bandwidth pass: a fixed grid of kGrid blocks streams every tensor with
+// 16-byte loads (4 in flight per thread), squares and sums each float4 in
+// fp32, accumulates those in fp64 per thread, reduces per block in a fixed
+// shuffle/shared-memory order and writes one fp64 partial per (launch, block,
+// class).  A one-block kernel then sums the partials in a fixed order, so the
+// result does not depend on scheduling.  Segments go to the kernel by value
+// (kSegsPerLaunch per launch), so no host->device copy is needed.
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kGrid = 1024;
+constexpr int kBlock = 256;
+constexpr int kSegsPerLaunch = 128;
+constexpr int kMaxSegs = 4096;
+
+struct ClipSeg {
+  const float* ptr;
+  int64_t len;
+  int32_t cls;  // 0 dense, 1 expert
+  int32_t pad;
+};
+struct ClipBatch {
+  ClipSeg seg[kSegsPerLaunch];
+  int32_t n;
+};
+
+__device__ __forceinline__ double block_sum(double v, double* s_red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < kBlock / 32; ++w) r += s_red[w];
+  __syncthreads();
+  return r;  // valid in thread 0
+}
+
+__device__ __forceinline__ float sq4(const float4& v) {
+  return v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+}
+
+__global__ void __launch_bounds__(kBlock) sumsq_kernel(const ClipBatch b, double* partials) {
+  __shared__ double s_red[kBlock / 32];
+  double acc[2] = {0.0, 0.0};
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x;
+  const int64_t nth = static_cast<int64_t>(gridDim.x) * kBlock;
+  for (int s = 0; s < b.n; ++s) {
+    const float* p = b.seg[s].ptr;
+    const int64_t n = b.seg[s].len;
+    const int64_t n4 = n >> 2;
+    const float4* p4 = reinterpret_cast<const float4*>(p);
+    double a = 0.0;
+    int64_t i = gtid;
+    for (; i + 3 * nth < n4; i += 4 * nth) {
+      const float4 v0 = __ldg(p4 + i);
+      const float4 v1 = __ldg(p4 + i + nth);
+      const float4 v2 = __ldg(p4 + i + 2 * nth);
+      const float4 v3 = __ldg(p4 + i + 3 * nth);
+      a += static_cast<double>(sq4(v0));
+      a += static_cast<double>(sq4(v1));
+      a += static_cast<double>(sq4(v2));
+      a += static_cast<double>(sq4(v3));
+    }
+    for (; i < n4; i += nth) a += static_cast<double>(sq4(__ldg(p4 + i)));
+    for (int64_t j = 4 * n4 + gtid; j < n; j += nth) {
+      const float v = __ldg(p + j);
+      a += static_cast<double>(v * v);
+    }
+    acc[b.seg[s].cls] += a;
+  }
+  const double d = block_sum(acc[0], s_red);
+  const double e = block_sum(acc[1], s_red);
+  if (threadIdx.x == 0) {
+    partials[2 * blockIdx.x] = d;
+    partials[2 * blockIdx.x + 1] = e;
+  }
+}
+
+__global__ void __launch_bounds__(kBlock) finish_kernel(const double* partials, int n_partials,
+                                                        int num_experts, double* out) {
+  __shared__ double s_red[kBlock / 32];
+  double a = 0.0, e = 0.0;
+  for (int i = threadIdx.x; i < n_partials; i += kBlock) {
+    a += partials[2 * i];
+    e += partials[2 * i + 1];
+  }
+  const double sd = block_sum(a, s_red);
+  const double ss = block_sum(e, s_red);
+  if (threadIdx.x == 0) {
+    out[0] = sqrt(sd + ss / static_cast<double>(num_experts));  // kappa^2 = 1/E
+    out[1] = sd;
+    out[2] = ss;
+  }
+}
+
+int64_t n_launches(int32_t n_dense, int32_t n_sparse) {
+  const int64_t n = static_cast<int64_t>(n_dense) + n_sparse;
+  return std::max<int64_t>(1, (n + kSegsPerLaunch - 1) / kSegsPerLaunch);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t sparseclip_workspace_size(int32_t n_dense, int32_t n_sparse) {
+  if (n_dense < 0 || n_sparse < 0 || static_cast<int64_t>(n_dense) + n_sparse > kMaxSegs) return 0;
+  return static_cast<size_t>(n_launches(n_dense, n_sparse)) * kGrid * 2 * sizeof(double);
+}
+
+extern "C" int32_t sparseclip_norm(const float* const* dense, const int64_t* dense_len,
+                                   int32_t n_dense, const float* const* sparse,
+                                   const int64_t* sparse_len, int32_t n_sparse,
+                                   int32_t num_experts, double* out, void* workspace,
+                                   size_t workspace_bytes, moe_stream_t stream) {
+  set_last_error("");
+  if (n_dense < 0 || n_sparse < 0 || static_cast<int64_t>(n_dense) + n_sparse > kMaxSegs)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: segment counts out of range");
+  if ((n_dense > 0 && (!dense || !dense_len)) || (n_sparse > 0 && (!sparse || !sparse_len)))
+    return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: null segment array");
+  if (num_experts < 1) return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: num_experts < 1");
+  if (!out) return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: null out");
+  const size_t need = sparseclip_workspace_size(n_dense, n_sparse);
+  if (!workspace || workspace_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "sparseclip_norm: workspace needs " + std::to_string(need) +
+                                       " bytes");
+  if (!aligned16(workspace)) return fail(MOE_ERR_ALIGNMENT, "sparseclip_norm: workspace");
+  std::vector<ClipSeg> segs;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int32_t n = pass == 0 ? n_dense : n_sparse;
+    const float* const* ptrs = pass == 0 ? dense : sparse;
+    const int64_t* lens = pass == 0 ? dense_len : sparse_len;
+    for (int32_t i = 0; i < n; ++i) {
+      if (lens[i] < 0) return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: negative length");
+      if (lens[i] == 0) continue;
+      if (!ptrs[i]) return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: null tensor");
+      if (!aligned16(ptrs[i])) return fail(MOE_ERR_ALIGNMENT, "sparseclip_norm: tensor not 16-byte aligned");
+      segs.push_back(ClipSeg{ptrs[i], lens[i], pass, 0});
+    }
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  double* partials = static_cast<double*>(workspace);
+  const int64_t launches = std::max<int64_t>(1, (static_cast<int64_t>(segs.size()) + kSegsPerLaunch - 1) / kSegsPerLaunch);
+  for (int64_t l = 0; l < launches; ++l) {
+    ClipBatch b{};
+    const size_t first = static_cast<size_t>(l) * kSegsPerLaunch;
+    b.n = static_cast<int32_t>(std::min<size_t>(kSegsPerLaunch, segs.size() - std::min(first, segs.size())));
+    for (int32_t i = 0; i < b.n; ++i) b.seg[i] = segs[first + i];
+    sumsq_kernel<<<kGrid, kBlock, 0, s>>>(b, partials + l * kGrid * 2);
+    int32_t rc = check_launch("sumsq_kernel");
+    if (rc != MOE_OK) return rc;
+  }
+  finish_kernel<<<1, kBlock, 0, s>>>(partials, static_cast<int>(launches * kGrid), num_experts, out);
+  return check_launch("finish_kernel");
+}

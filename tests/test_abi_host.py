@@ -1,0 +1,121 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+the header declares, and its host-side queries and argument validation
+behave as documented (a rejected call returns before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**\s*((?:moe|sparseclip)_\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import sparse_mixture_experts_fwd_b200 as m
+    return m
+
+
+def test_every_declared_symbol_is_exported(moe):
+    names = declared_functions()
+    assert len(names) >= 18, names
+    raw = ctypes.CDLL(moe.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in moe_b200.h but not exported"
+    assert set(names) == set(moe.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_struct_layout(moe):
+    assert moe.lib.moe_abi_version() == 1
+    assert moe.lib.moe_config_size() == 48 == ctypes.sizeof(moe.MoEConfig)
+    assert moe.lib.moe_workspace_map_size() == ctypes.sizeof(moe.WorkspaceMap)
+
+
+def test_capacity_eq3(moe):
+    # Switch notes sec. 2.2 eq. (3) at the five workloads, and the floor reading
+    assert [moe.capacity(T, E, cf) for T, E, cf in
+            [(256, 8, 1.0), (8192, 128, 1.25), (16384, 64, 2.0), (32768, 64, 1.25),
+             (65536, 256, 1.0)]] == [32, 80, 512, 640, 256]
+    assert moe.capacity(10, 3, 1.0) == 3
+    assert moe.capacity(10, 0, 1.0) == -1
+    assert moe.capacity(-1, 2, 1.0) == -1
+
+
+def cfg(moe, **kw):
+    base = dict(T=8192, d_model=768, d_ff=3072, E=128, k=1, capacity_=80)
+    base.update(kw)
+    import torch
+    dtype = base.pop("dtype", torch.bfloat16)
+    return moe.make_config(base.pop("T"), base.pop("d_model"), base.pop("d_ff"), base.pop("E"),
+                           base.pop("k"), base.pop("capacity_"), dtype=dtype, **base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(E=0), -1), (dict(E=512), -2), (dict(k=3), -2), (dict(k=2, E=1), -1),
+    (dict(capacity_=-1), -1), (dict(d_model=100), -2), (dict(E=40), -2),
+    (dict(mode="rre", k=2, num_groups=8), -1), (dict(mode="rre", num_groups=3), -1),
+    (dict(T=-5), -1),
+])
+def test_config_rejections(moe, kw, code):
+    c = cfg(moe, **kw)
+    assert moe.lib.moe_config_check(ctypes.byref(c)) == code
+    assert moe.lib.moe_last_error().decode() != ""
+    assert moe.lib.moe_workspace_size(ctypes.byref(c)) == 0
+
+
+def test_config_accepts_workloads(moe):
+    import torch
+    import synth
+    for w in synth.WORKLOADS.values():
+        C = moe.capacity(w.T, w.E, w.capacity_factor)
+        c = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, C, dtype=w.torch_dtype, mode=w.mode,
+                            num_groups=w.num_groups, seed=w.seed)
+        assert moe.lib.moe_config_check(ctypes.byref(c)) == 0, w.name
+        m = moe.workspace_layout(c)
+        es = 2 if w.dtype == "bf16" else 4
+        offs = [m.logits, m.expert_idx, m.gate, m.slot, m.kept, m.tok_of_row, m.arrivals,
+                m.kept_cnt, m.n_dropped, m.scratch, m.xe, m.H, m.ye, m.total]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert m.total - m.ye >= w.E * C * w.d_model * es
+        assert m.ye - m.H >= w.E * C * w.d_ff * es
+
+
+def test_calls_rejected_on_host(moe):
+    import torch  # noqa: F401
+    c = cfg(moe)
+    p = ctypes.c_void_p(4096)  # aligned dummy, never dereferenced: validation fails first
+    # null x
+    assert moe.lib.moe_router(ctypes.byref(c), None, p, None, p, None, None) == -1
+    # misaligned logits
+    assert moe.lib.moe_router(ctypes.byref(c), p, p, None, ctypes.c_void_p(4100), None, None) == -3
+    # workspace too small
+    assert moe.lib.moe_layer_forward(ctypes.byref(c), p, p, None, None, p, p, p, p, 10, None, None) == -4
+    # topk_assign without workspace
+    assert moe.lib.moe_topk_assign(ctypes.byref(c), p, None, p, p, p, p, p, p, p, p, None, 0,
+                                   None, None) == -4
+    # invalid config reaches no launch
+    bad = cfg(moe, k=3)
+    assert moe.lib.moe_expert_ffn(ctypes.byref(bad), p, p, p, p, p, p, None, None) == -2
+    assert moe.lib.moe_dispatch(None, p, p, p, p, p, None) == -1
+    # sparseclip
+    assert moe.lib.sparseclip_norm(None, None, 0, None, None, 0, 0, p, p, 1 << 20, None) == -1
+    assert moe.lib.sparseclip_workspace_size(1, 64) == 1024 * 2 * 8
+    assert moe.lib.sparseclip_workspace_size(-1, 0) == 0
+
+
+def test_library_refuses_cpu_tensors(moe):
+    import torch
+    c = cfg(moe, T=4, d_model=64, d_ff=64, E=16, capacity_=1)
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        moe.router(c, x, torch.zeros(16, 64, dtype=torch.bfloat16),
+                   logits=torch.zeros(4, 16))

@@ -1,0 +1,412 @@
+"""GPU parity: every C-ABI call against the CPU oracle on the same seeded inputs.
+
+Bar (per call):
+  * expert choice, slots, drop masks, row->token map and counts: bit-exact
+    when both sides start from the same fp32 logits;
+  * end to end, a token may route differently only if its sorted top-(k+1)
+    oracle logits have an adjacent gap below 1e-5, and the slots must then
+    equal the oracle's assignment of the GPU's choices bit-exactly;
+  * gates and the SparseClip norm: relative 1e-5;
+  * bf16 activations: |gpu - ref| <= 2e-2 + 1e-2 |ref| per element, plus
+    tighter arithmetic bounds where the arithmetic fixes one.
+"""
+import concurrent.futures as cf
+import math
+
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import (ATOL, GATE_RTOL, RTOL, assert_close, margin_exempt, threads, to_dev,
+                         workload_case)
+
+pytestmark = pytest.mark.gpu
+
+ALL = ["tiny_switch", "switch_base", "xmoe_top2", "pangu_rre", "skewed_switch"]
+TOPK = ["tiny_switch", "switch_base", "xmoe_top2", "skewed_switch"]
+
+
+@pytest.fixture(scope="module")
+def moe(cuda_device):
+    import sparse_mixture_experts_fwd_b200 as m
+    return m
+
+
+class Case:
+    """One workload: CPU inputs, the oracle's routing reference, device copies."""
+
+    def __init__(self, moe, name, dev):
+        self.name = name
+        self.w, self.inp, self.ref = workload_case(name)
+        self.C = self.ref["C"]
+        self.cfg = make_cfg(moe, self.w, self.C)
+        self.dev = {k: to_dev(v, dev) for k, v in self.inp.items()}
+
+
+@pytest.fixture(scope="module", params=ALL)
+def case(moe, cuda_device, request):
+    c = Case(moe, request.param, cuda_device)
+    yield c
+    del c.dev
+    torch.cuda.empty_cache()
+
+
+def make_cfg(moe, w, C, T=None):
+    return moe.make_config(w.T if T is None else T, w.d_model, w.d_ff, w.E, w.k, C,
+                           dtype=w.torch_dtype, mode=w.mode, num_groups=w.num_groups, seed=w.seed)
+
+
+def zero_status(dev):
+    return torch.zeros(1, dtype=torch.int32, device=dev)
+
+
+# ---------------------------------------------------------------------------
+# a1 router
+# ---------------------------------------------------------------------------
+
+def test_router_logits(moe, cuda_device, case):
+    w, inp, ref, D = case.w, case.inp, case.ref, case.dev
+    if w.mode != "topk":
+        pytest.skip("RRE has no router")
+    dev = cuda_device
+    cfg = case.cfg
+    st = zero_status(dev)
+    got = moe.router(cfg, D["x"], D["Wr"], D["bias"], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    got = got.cpu().double()
+    r = ref["logits"].double()
+    # fp32 accumulation of d exact products: |err| <= 2 d u sum|x w| (+ final rounding)
+    absdot = inp["x"].double().abs() @ inp["Wr"].double().abs().T
+    u = 2.0 ** -24
+    bound = 2 * w.d_model * u * absdot + 2 * u * r.abs() + 1e-30
+    err = (got - r).abs()
+    assert bool((err <= bound).all()), f"max err {err.max():.3e}"
+    assert float(err.max()) < 1e-4
+
+
+# ---------------------------------------------------------------------------
+# a2-a4 gate, top-k / RRE, capacity assignment (bit-exact on identical logits)
+# ---------------------------------------------------------------------------
+
+def test_assign_bitexact(moe, cuda_device, case):
+    w, inp, ref, D = case.w, case.inp, case.ref, case.dev
+    dev = cuda_device
+    cfg = case.cfg
+    st = zero_status(dev)
+    if w.mode == "topk":
+        out = moe.topk_assign(cfg, logits=ref["logits"].to(dev), status=st)
+    else:
+        out = moe.topk_assign(cfg, domain_id=D["domain"], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for key in ("expert_idx", "slot", "kept", "arrivals", "kept_cnt"):
+        assert torch.equal(out[key].cpu(), ref[key]), key
+    C = ref["C"]
+    assert torch.equal(out["tok_of_row"].cpu()[: w.E * C], ref["tok_of_row"])
+    assert int(out["n_dropped"].item()) == ref["n_dropped"]
+    g, rg = out["gate"].cpu().double(), ref["gate"].double()
+    assert bool(((g - rg).abs() <= GATE_RTOL * rg.abs()).all())
+
+
+def test_assign_ties_and_hot_expert(moe, cuda_device):
+    """Integer logits with many exact ties, k = 1 and 2, capacities around the load."""
+    dev = cuda_device
+    gen = torch.Generator().manual_seed(11)
+    for k in (1, 2):
+        for T, E, C in [(5000, 16, 200), (3001, 64, 0), (2048, 256, 3), (1, 16, 1), (777, 32, 777)]:
+            logits = torch.randint(-3, 4, (T, E), generator=gen).float()
+            logits[:, 5] += 2.0  # a hot expert
+            cfg = moe.make_config(T, 64, 64, E, k, C, dtype=torch.bfloat16)
+            out = moe.topk_assign(cfg, logits=logits.to(dev))
+            idx, gate = oracle.gate_topk(logits, k)
+            a = oracle.assign(idx, E, C)
+            torch.cuda.synchronize()
+            assert torch.equal(out["expert_idx"].cpu(), idx)
+            for key in ("slot", "kept", "arrivals", "kept_cnt"):
+                assert torch.equal(out[key].cpu(), a[key]), (k, T, E, C, key)
+            assert torch.equal(out["tok_of_row"].cpu()[: E * C], a["tok_of_row"])
+            assert int(out["n_dropped"].item()) == a["n_dropped"]
+            assert bool(((out["gate"].cpu().double() - gate.double()).abs()
+                         <= GATE_RTOL * gate.double()).all())
+
+
+def test_rre_bad_domain_reported(moe, cuda_device):
+    dev = cuda_device
+    cfg = moe.make_config(64, 64, 64, 16, 1, 8, dtype=torch.bfloat16, mode="rre", num_groups=4)
+    dom = torch.zeros(64, dtype=torch.int32)
+    dom[7] = 9  # outside 0..3
+    st = zero_status(dev)
+    out = moe.topk_assign(cfg, domain_id=dom.to(dev), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & moe.STATUS_BAD_DOMAIN
+    assert 0 <= int(out["expert_idx"][7, 0]) < 4
+
+
+# ---------------------------------------------------------------------------
+# a5 dispatch, a7 combine
+# ---------------------------------------------------------------------------
+
+def test_dispatch_bitexact(moe, cuda_device, case):
+    w, inp, ref, D = case.w, case.inp, case.ref, case.dev
+    dev = cuda_device
+    C = case.C
+    cfg = case.cfg
+    xe = moe.dispatch(cfg, D["x"], ref["expert_idx"].to(dev), ref["slot"].to(dev),
+                      ref["kept"].to(dev))
+    torch.cuda.synchronize()
+    xe_ref = oracle.dispatch(inp["x"], ref["tok_of_row"], ref["kept_cnt"], w.E, C)
+    xe = xe.cpu()
+    for e in range(w.E):
+        n = int(ref["kept_cnt"][e])
+        assert torch.equal(xe[e, :n].view(torch.int16) if w.dtype == "bf16" else xe[e, :n],
+                           xe_ref[e, :n].view(torch.int16) if w.dtype == "bf16" else xe_ref[e, :n]), e
+
+
+def test_combine(moe, cuda_device, case):
+    w, inp, ref = case.w, case.inp, case.ref
+    dev = cuda_device
+    C = case.C
+    cfg = case.cfg
+    ye = synth.normal(w.seed, 99, (w.E, C, w.d_model), 0.5, w.torch_dtype)
+    y = moe.combine(cfg, ye.to(dev), ref["expert_idx"].to(dev), ref["gate"].to(dev),
+                    ref["slot"].to(dev), ref["kept"].to(dev))
+    torch.cuda.synchronize()
+    y_ref = oracle.combine(ye, ref["expert_idx"], ref["gate"], ref["slot"], ref["kept"], w.T)
+    # fp32 accumulation then one rounding vs exact then one rounding: at most one ulp apart
+    ulp = 2.0 ** -7 if w.dtype == "bf16" else 2.0 ** -22
+    assert_close(y.cpu(), y_ref, atol=1e-37, rtol=ulp, what="combine")
+    none_kept = ref["kept"].sum(1) == 0
+    assert bool((y.cpu()[none_kept] == 0).all())
+
+
+# ---------------------------------------------------------------------------
+# a6 expert FFN
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_expert_ffn_ragged_tiles(moe, cuda_device, dtype):
+    """Several 128-row and 256-column tiles, ragged kept counts, C not a tile multiple."""
+    dev = cuda_device
+    E, C, d, f = 5, 300, 256, 768
+    kept = torch.tensor([300, 0, 129, 1, 128], dtype=torch.int32)
+    xe = synth.normal(21, 1, (E, C, d), 1.0, dtype)
+    W1 = synth.normal(21, 3, (E, f, d), 0.02, dtype)
+    W2 = synth.normal(21, 4, (E, d, f), 0.02, dtype)
+    cfg = moe.make_config(1, d, f, E, 1, C, dtype=dtype)
+    sentinel = float("nan")
+    H = torch.full((E, C, f), sentinel, dtype=dtype, device=dev)
+    ye = torch.full((E, C, d), sentinel, dtype=dtype, device=dev)
+    st = zero_status(dev)
+    moe.expert_ffn(cfg, xe.to(dev), W1.to(dev), W2.to(dev), kept.to(dev), H=H, ye=ye, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ye_ref, H_ref = oracle.expert_ffn(xe, W1, W2, kept, with_H=True, nthreads=threads())
+    H, ye = H.cpu(), ye.cpu()
+    for e in range(E):
+        n = int(kept[e])
+        if dtype == torch.bfloat16:
+            assert_close(H[e, :n], H_ref[e, :n], what=f"H[{e}]")
+            assert_close(ye[e, :n], ye_ref[e, :n], what=f"ye[{e}]")
+            # beyond the stated tolerance: rounding differences only, rarely more than 1 ulp
+            for a, b in ((H[e, :n], H_ref[e, :n]), (ye[e, :n], ye_ref[e, :n])):
+                if a.numel():
+                    far = (a.double() - b.double()).abs() > 2.0 ** -7 * b.double().abs() + 1e-3
+                    assert float(far.double().mean()) < 1e-3
+        else:
+            assert_close(H[e, :n], H_ref[e, :n], atol=1e-5, rtol=1e-5, what=f"H[{e}]")
+            assert_close(ye[e, :n], ye_ref[e, :n], atol=1e-5, rtol=1e-5, what=f"ye[{e}]")
+        # rows past kept_cnt are never written
+        assert bool(torch.isnan(H[e, n:].float()).all()) and bool(torch.isnan(ye[e, n:].float()).all())
+
+
+# ---------------------------------------------------------------------------
+# the whole layer at full size, sampled outputs
+# ---------------------------------------------------------------------------
+
+def _sample_tokens(ref, T, k, n_random=64):
+    g = torch.Generator().manual_seed(5)
+    picks = list(range(min(16, T))) + list(range(max(0, T - 16), T))
+    picks += torch.randint(0, T, (n_random,), generator=g).tolist()
+    kept_n = ref["kept"].sum(1)
+    picks += torch.nonzero(kept_n == 0).flatten()[:8].tolist()
+    if k == 2:
+        picks += torch.nonzero(kept_n == 1).flatten()[:8].tolist()
+    return sorted(set(picks))
+
+
+def test_layer_forward_full(moe, cuda_device, case):
+    w, inp, ref, D = case.w, case.inp, case.ref, case.dev
+    dev = cuda_device
+    C = case.C
+    cfg = case.cfg
+    ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    st = zero_status(dev)
+    y = moe.layer_forward(cfg, D["x"], D["W1"], D["W2"], Wr=D["Wr"], bias=D["bias"],
+                          domain_id=D["domain"], workspace=ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    v = {k_: t.cpu() for k_, t in moe.workspace_views(cfg, ws).items()}
+    y = y.cpu()
+    gidx = v["expert_idx"]
+    if w.mode == "topk":
+        exempt = margin_exempt(ref["logits"], w.k)
+        differs = (gidx != ref["expert_idx"]).any(1)
+        assert not bool((differs & ~exempt).any()), "routing differs on a token with a clear margin"
+        same = ~differs
+        g, rg = v["gate"][same].double(), ref["gate"][same].double()
+        assert bool(((g - rg).abs() <= GATE_RTOL * rg.abs()).all())
+    else:
+        assert torch.equal(gidx, ref["expert_idx"])
+        differs = torch.zeros(w.T, dtype=torch.bool)
+    # the slot assignment of the GPU's own choices is the oracle's, bit for bit
+    a = oracle.assign(gidx, w.E, C)
+    for key in ("slot", "kept", "arrivals", "kept_cnt"):
+        assert torch.equal(v[key], a[key]), key
+    assert int(v["n_dropped"].item()) == a["n_dropped"]
+    # outputs of sampled tokens, each computed alone by the oracle
+    toks = [t for t in _sample_tokens(a, w.T, w.k) if not bool(differs[t])]
+    gate_src = ref["gate"]
+
+    def one(t):
+        return oracle.token_forward(inp["x"][t], inp["W1"], inp["W2"], gidx[t], gate_src[t], a["kept"][t])
+
+    with cf.ThreadPoolExecutor(max_workers=threads()) as ex:
+        y_ref = list(ex.map(one, toks))
+    for t, yr in zip(toks, y_ref):
+        assert_close(y[t], yr, what=f"y[{t}]")
+        if int(a["kept"][t].sum()) == 0:
+            assert bool((y[t] == 0).all())
+    # expert outputs of sampled kept rows against the oracle's expert alone
+    rows = []
+    for t in toks[:24]:
+        for j in range(w.k):
+            if a["kept"][t, j]:
+                rows.append((t, int(gidx[t, j]), int(a["slot"][t, j])))
+
+    def one_row(r):
+        t, e, s = r
+        return oracle.expert_row(inp["x"][t], inp["W1"][e], inp["W2"][e])
+
+    with cf.ThreadPoolExecutor(max_workers=threads()) as ex:
+        ye_ref = list(ex.map(one_row, rows))
+    for (t, e, s), yr in zip(rows, ye_ref):
+        assert_close(v["ye"][e, s], yr, what=f"ye[{e},{s}]")
+        assert torch.equal(v["xe"][e, s].view(torch.int16) if w.dtype == "bf16" else v["xe"][e, s],
+                           inp["x"][t].view(torch.int16) if w.dtype == "bf16" else inp["x"][t])
+
+
+def test_layer_forward_deterministic(moe, cuda_device, case):
+    D = case.dev
+    kw = dict(Wr=D["Wr"], bias=D["bias"], domain_id=D["domain"])
+    y1 = moe.layer_forward(case.cfg, D["x"], D["W1"], D["W2"], **kw)
+    y2 = moe.layer_forward(case.cfg, D["x"], D["W1"], D["W2"], **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int32 if case.w.dtype == "f32" else torch.int16),
+                       y2.view(torch.int32 if case.w.dtype == "f32" else torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# small whole-layer cases: every intermediate against the oracle's layer
+# ---------------------------------------------------------------------------
+
+SMALL = [
+    # name, T, d, f, E, k, cf, mode, G, hot_bias
+    ("ragged_top2", 1000, 128, 256, 16, 2, 1.0, "topk", 1, 0.0),
+    ("few_tokens", 5, 64, 128, 16, 1, 1.0, "topk", 1, 0.0),
+    ("one_hot_expert", 700, 64, 192, 32, 1, 1.0, "topk", 1, 100.0),
+    ("many_experts_top2", 900, 64, 128, 256, 2, 4.0, "topk", 1, 0.0),
+    ("rre_small", 1500, 128, 256, 32, 1, 1.25, "rre", 4, 0.0),
+    ("zero_capacity", 300, 64, 64, 16, 1, 0.0, "topk", 1, 0.0),
+    ("tiny_fp32_top2", 400, 32, 48, 8, 2, 1.5, "topk", 1, 0.0),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_layer_small_cases(moe, cuda_device, case):
+    name, T, d, f, E, k, cf_, mode, G, hot = case
+    dev = cuda_device
+    dtype = "f32" if "fp32" in name else "bf16"
+    w = synth.Workload(name, T=T, d_model=d, d_ff=f, E=E, k=k, capacity_factor=cf_, dtype=dtype,
+                       mode=mode, num_groups=G, hot_experts=1 if hot else 0, hot_bias=hot, seed=3)
+    inp = synth.layer_inputs(w)
+    C = oracle.capacity(T, E, cf_)
+    r = oracle.layer_forward(inp["x"], inp["W1"], inp["W2"], E=E, k=k, C=C, Wr=inp["Wr"],
+                             bias=inp["bias"], domain=inp["domain"], G=G, seed=w.seed, with_H=True,
+                             nthreads=threads())
+    cfg = make_cfg(moe, w, C)
+    ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    st = zero_status(dev)
+    y = moe.layer_forward(cfg, inp["x"].to(dev), inp["W1"].to(dev), inp["W2"].to(dev),
+                          Wr=to_dev(inp["Wr"], dev), bias=to_dev(inp["bias"], dev),
+                          domain_id=to_dev(inp["domain"], dev), workspace=ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    v = {k_: t.cpu() for k_, t in moe.workspace_views(cfg, ws).items()}
+    if mode == "topk":
+        exempt = margin_exempt(r["logits"], k)
+        differs = (v["expert_idx"] != r["expert_idx"]).any(1)
+        assert not bool((differs & ~exempt).any())
+        assert not bool(differs.any()), "small cases are expected to route identically"
+    for key in ("expert_idx", "slot", "kept", "arrivals", "kept_cnt"):
+        assert torch.equal(v[key], r[key]), key
+    assert int(v["n_dropped"].item()) == r["n_dropped"]
+    if hot:
+        assert int(v["arrivals"][0]) == T and int(v["kept_cnt"][0]) == min(T, C)
+    if C == 0:
+        assert int(v["n_dropped"].item()) == T * k
+    tol = dict(atol=1e-5, rtol=1e-5) if dtype == "f32" else {}
+    assert_close(y.cpu(), r["y"], what="y", **tol)
+    for e in range(E):
+        n = int(r["kept_cnt"][e])
+        assert_close(v["H"][e, :n], r["H"][e, :n], what=f"H[{e}]", **tol)
+        assert_close(v["ye"][e, :n], r["ye"][e, :n], what=f"ye[{e}]", **tol)
+
+
+def test_layer_zero_tokens(moe, cuda_device):
+    dev = cuda_device
+    cfg = moe.make_config(0, 64, 64, 16, 1, 0, dtype=torch.bfloat16)
+    x = torch.empty(0, 64, dtype=torch.bfloat16, device=dev)
+    W = torch.zeros(16, 64, 64, dtype=torch.bfloat16, device=dev)
+    Wr = torch.zeros(16, 64, dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(max(256, moe.workspace_size(cfg)), dtype=torch.uint8, device=dev)
+    y = moe.layer_forward(cfg, x, W, W, Wr=Wr, workspace=ws)
+    torch.cuda.synchronize()
+    assert y.shape == (0, 64)
+    v = moe.workspace_views(cfg, ws)
+    assert int(v["n_dropped"].item()) == 0 and int(v["arrivals"].sum()) == 0
+
+
+# ---------------------------------------------------------------------------
+# a8 SparseClip norm
+# ---------------------------------------------------------------------------
+
+def test_sparseclip_full(moe, cuda_device):
+    w = synth.WORKLOADS["xmoe_top2"]
+    dense, sparse = synth.sparseclip_inputs(w)
+    dev = cuda_device
+    out = moe.sparseclip_norm([t.to(dev) for t in dense], [t.to(dev) for t in sparse], w.E)
+    torch.cuda.synchronize()
+    ref = oracle.sparseclip_norm(dense, sparse, w.E)
+    got = out.cpu().tolist()
+    assert abs(got[0] - ref) <= GATE_RTOL * ref, (got[0], ref)
+    ref_d = oracle.sparseclip_norm(dense, [torch.zeros(4)], w.E)
+    assert abs(got[1] - ref_d ** 2) <= GATE_RTOL * ref_d ** 2
+    assert math.isclose(got[0], math.sqrt(got[1] + got[2] / 64), rel_tol=1e-12)
+
+
+def test_sparseclip_segments_and_tails(moe, cuda_device):
+    dev = cuda_device
+    dense = [synth.normal(1, 6, (n,), 1e-3, torch.float32) for n in (1, 3, 4097, 0, 100_003)]
+    sparse = [synth.normal(1, 7 + 16 * s, (513 + 7 * s,), 1e-3, torch.float32) for s in range(300)]
+    for E in (1, 64, 7):
+        out = moe.sparseclip_norm([t.to(dev) for t in dense], [t.to(dev) for t in sparse], E)
+        torch.cuda.synchronize()
+        ref = oracle.sparseclip_norm(dense, sparse, E)
+        assert abs(out[0].item() - ref) <= GATE_RTOL * ref, (E, out[0].item(), ref)
+    # hand-worked example: sqrt(50)
+    out = moe.sparseclip_norm([torch.tensor([3.0, 4.0], device=dev)],
+                              [torch.tensor([6.0, 8.0], device=dev)], 4)
+    torch.cuda.synchronize()
+    assert abs(out[0].item() - math.sqrt(50.0)) < 1e-12

@@ -288,6 +288,19 @@ def test_layer_forward_is_composition_of_steps(oracle_lib):
     assert int(a["kept"].sum()) + a["n_dropped"] == w.T
 
 
+def test_token_forward_matches_layer(oracle_lib):
+    w = synth.WORKLOADS["xmoe_top2"].scaled(T=300, d_model=128, d_ff=256, E=8)
+    inp = synth.layer_inputs(w)
+    C = oracle.capacity(w.T, w.E, w.capacity_factor)
+    r = oracle.layer_forward(inp["x"], inp["W1"], inp["W2"], E=w.E, k=2, C=C, Wr=inp["Wr"])
+    partly = [t for t in range(w.T) if int(r["kept"][t].sum()) == 1]
+    assert partly, "expected a token with one of two choices dropped"
+    for t in list(range(0, w.T, 23)) + partly[:5]:
+        y = oracle.token_forward(inp["x"][t], inp["W1"], inp["W2"], r["expert_idx"][t],
+                                 r["gate"][t], r["kept"][t])
+        assert torch.equal(y, r["y"][t])
+
+
 def test_rre_layer_has_unit_gates(oracle_lib):
     w = synth.WORKLOADS["pangu_rre"].scaled(T=512, d_model=64, d_ff=128)
     inp = synth.layer_inputs(w)
