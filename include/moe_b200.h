@@ -131,7 +131,7 @@ size_t sparseclip_workspace_size(int32_t n_dense, int32_t n_sparse);
  *   logits[t, e] = sum_c x[t, c] * Wr[e, c] (+ bias[e])
  * x [T, d] and Wr [E, d] in cfg->dtype; bias [E] fp32, nullable; logits
  * [T, E] fp32.  bf16 inputs: exact products, fp32 accumulation on the
- * tensor cores (requires E % 16 == 0).  fp32 inputs: fp32 FMA chain. */
+ * tensor cores.  fp32 inputs: fp32 FMA chain. */
 int32_t moe_router(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
                    float* logits, int32_t* status, moe_stream_t stream);
 

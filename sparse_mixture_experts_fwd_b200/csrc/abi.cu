@@ -66,8 +66,6 @@ int32_t check_cfg(const moe_config* c) {
   if (c->dtype == MOE_DTYPE_BF16) {
     if (c->d_model % 64 || c->d_ff % 64)
       return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d_model and d_ff multiples of 64");
-    if (c->mode == MOE_ROUTE_TOPK && c->E % 16)
-      return fail(MOE_ERR_UNSUPPORTED, "bf16 router needs E multiple of 16");
   } else {
     if (c->d_model % 4 || c->d_ff % 4)
       return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d_model and d_ff multiples of 4");
@@ -193,10 +191,7 @@ int32_t moe_router(const moe_config* cfg, const void* x, const void* Wr, const f
   MOE_TRY(need_ptr(bias, "bias", false));
   MOE_TRY(need_ptr(logits, "logits"));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cfg->dtype == MOE_DTYPE_BF16) {
-    if (cfg->E % 16) return fail(MOE_ERR_UNSUPPORTED, "bf16 router needs E multiple of 16");
-    return launch_router_tc(*cfg, x, Wr, bias, logits, status, s);
-  }
+  if (cfg->dtype == MOE_DTYPE_BF16) return launch_router_tc(*cfg, x, Wr, bias, logits, status, s);
   return launch_router_f32(*cfg, x, Wr, bias, logits, s);
 }
 

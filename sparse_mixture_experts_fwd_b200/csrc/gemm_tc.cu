@@ -247,15 +247,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           dev::tmem_wait_ld();
           const int n = n0 + c * 16;
           if (row_ok && n < p.N) {
-            float v[16];
+            if (n + 16 <= p.N && (p.out_ld & 3) == 0) {
+              float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              v[i] = __uint_as_float(r[i]);
-              if (p.bias) v[i] += __ldg(p.bias + n + i);
+              for (int i = 0; i < 16; ++i) {
+                v[i] = __uint_as_float(r[i]);
+                if (p.bias) v[i] += __ldg(p.bias + n + i);
+              }
+              float4* dst = reinterpret_cast<float4*>(out + n);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {  // ragged last columns or rows not 16-byte aligned
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (n + i < p.N) out[n + i] = __uint_as_float(r[i]) + (p.bias ? __ldg(p.bias + n + i) : 0.f);
             }
-            float4* dst = reinterpret_cast<float4*>(out + n);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
       } else {

@@ -61,7 +61,7 @@ def cfg(moe, **kw):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(E=0), -1), (dict(E=512), -2), (dict(k=3), -2), (dict(k=2, E=1), -1),
-    (dict(capacity_=-1), -1), (dict(d_model=100), -2), (dict(E=40), -2),
+    (dict(capacity_=-1), -1), (dict(d_model=100), -2), (dict(d_ff=96), -2),
     (dict(mode="rre", k=2, num_groups=8), -1), (dict(mode="rre", num_groups=3), -1),
     (dict(T=-5), -1),
 ])
