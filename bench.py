@@ -33,6 +33,7 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+METRIC = "MoE-layer tokens/sec (1 B200); expert-FFN TFLOP/s; dispatch+combine GB/s"
 
 
 def parse():
@@ -66,15 +67,15 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
         self.proc = None
         self.lines = []
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
@@ -167,7 +168,7 @@ def oracle_step_fn(w, T_s):
 
 def size_oracle_sample(w, seconds):
     """Pick a token count whose oracle step takes about `seconds`."""
-    T_s = 32
+    T_s = min(w.T, max(64, int(4 * w.E / w.capacity_factor) + 1))  # capacity >= 4 in the probe
     step, _ = oracle_step_fn(w, T_s)
     t0 = time.perf_counter()
     step()
@@ -198,7 +199,7 @@ def run_reference(args, w, world, rank):
         step()
     dt = time.perf_counter() - t0
     value = T_s * args.steps / dt
-    out = {"impl": "reference", "metric": "MoE-layer tokens/sec", "value": value,
+    out = {"impl": "reference", "metric": METRIC, "value": value,
            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -286,7 +287,21 @@ def run_b200(args, w, world, rank, local):
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    with ClockSampler(gpu_id) as clk:
+        # untimed pre-roll so the clock samples cover at least 1.5 s under this load
+        t_end = time.perf_counter() + 1.5
+        i = 0
+        with torch.cuda.stream(stream):
+            while time.perf_counter() < t_end:
+                step(i)
+                i += 1
+                if i % 32 == 0:
+                    stream.synchronize()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 step(args.warmup + i, evs[i])
@@ -372,7 +387,7 @@ def run_b200(args, w, world, rank, local):
         return
     clocks = clk.summary()
     out = {
-        "metric": "MoE-layer tokens/sec (1 B200); expert-FFN TFLOP/s; dispatch+combine GB/s",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
