@@ -206,6 +206,30 @@ int32_t sparseclip_norm(const float* const* dense, const int64_t* dense_len, int
                         int32_t num_experts, double* out, void* workspace, size_t workspace_bytes,
                         moe_stream_t stream);
 
+/* sparseclip_norm without a workspace, for callers that cannot allocate
+ * device memory: a runtime whose HBM is handed out once at start-up by its
+ * own pool and that forbids allocation afterwards, or code that must not call
+ * the CUDA allocator where it runs (allocator callbacks, out-of-memory
+ * recovery).  The pages describe no such entry point; it has no counterpart
+ * there.  Same arguments and result as sparseclip_norm minus the workspace.
+ * The partial sums live in a fixed 128 KiB array inside the library's own
+ * device memory, present on every GPU that loads the library until the
+ * process exits.  Limits and behaviour:
+ *   * n_dense + n_sparse <= 1024, else MOE_ERR_UNSUPPORTED (nothing launched);
+ *   * the first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture;
+ *   * the call allocates nothing (no cudaMalloc/cudaFree, no allocating
+ *     library routine);
+ *   * every call on a device shares the array: calls that overlap on the
+ *     GPU (other streams or host threads) race, so the caller serialises
+ *     them.  Each call writes every partial it reads, so no clearing is
+ *     needed between calls. */
+int32_t sparseclip_norm_noalloc(const float* const* dense, const int64_t* dense_len,
+                                int32_t n_dense, const float* const* sparse,
+                                const int64_t* sparse_len, int32_t n_sparse, int32_t num_experts,
+                                double* out, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

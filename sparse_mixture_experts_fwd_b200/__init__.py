@@ -65,6 +65,7 @@ SIGNATURES = {
     "moe_combine": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "moe_layer_forward": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp], _i32),
     "sparseclip_norm": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
+    "sparseclip_norm_noalloc": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
 }
 
 

@@ -166,3 +166,105 @@ extern "C" int32_t sparseclip_norm(const float* const* dense, const int64_t* den
   finish_kernel<<<1, kBlock, 0, s>>>(partials, static_cast<int>(launches * kGrid), num_experts, out);
   return check_launch("finish_kernel");
 }
+
+// ---------------------------------------------------------------------------
+// No-allocation variant.
+//
+// Some callers cannot hand the library a workspace: a process whose device
+// memory is carved up once at start-up by its own pool (a serving or
+// training runtime that forbids allocation on its hot path), or code running
+// where calling the CUDA allocator is not allowed or would interfere with
+// the caller's allocator (allocator callbacks, out-of-memory recovery).
+// sparseclip_norm_noalloc keeps its per-block partial sums in a fixed array
+// in the library's own device memory instead.  The array is 128 KiB and
+// exists on every GPU that loads the library until the process exits; it
+// bounds the call to kStaticMaxSegs tensors.  Every call writes each partial
+// it later reads, so nothing needs clearing between calls, but all calls on a
+// device share the array: calls that overlap on the GPU (other streams,
+// other host threads) race and must be serialised by the caller.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace moe {
+namespace {
+
+constexpr int kStaticMaxSegs = 1024;
+constexpr int kStaticMaxLaunches = kStaticMaxSegs / kSegsPerLaunch;
+
+static __device__ __align__(256) double g_static_partials[kStaticMaxLaunches * kGrid * 2];
+
+std::mutex g_static_mu;
+double* g_static_ptr[64] = {};
+
+// Device address of g_static_partials on the current device, looked up once
+// per device (with that device current) on the first call made there.
+int32_t static_partials(double** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal >= 64");
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_partials);
+    if (e != cudaSuccess || !p)
+      return fail(MOE_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    g_static_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int32_t sparseclip_norm_noalloc(const float* const* dense, const int64_t* dense_len,
+                                           int32_t n_dense, const float* const* sparse,
+                                           const int64_t* sparse_len, int32_t n_sparse,
+                                           int32_t num_experts, double* out, moe_stream_t stream) {
+  set_last_error("");
+  if (n_dense < 0 || n_sparse < 0)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm_noalloc: negative segment count");
+  if (static_cast<int64_t>(n_dense) + n_sparse > kStaticMaxSegs)
+    return fail(MOE_ERR_UNSUPPORTED, "sparseclip_norm_noalloc: at most " +
+                                         std::to_string(kStaticMaxSegs) +
+                                         " tensors (n_dense + n_sparse) per call");
+  if ((n_dense > 0 && (!dense || !dense_len)) || (n_sparse > 0 && (!sparse || !sparse_len)))
+    return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm_noalloc: null segment array");
+  if (num_experts < 1)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm_noalloc: num_experts < 1");
+  if (!out) return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm_noalloc: null out");
+  std::vector<ClipSeg> segs;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int32_t n = pass == 0 ? n_dense : n_sparse;
+    const float* const* ptrs = pass == 0 ? dense : sparse;
+    const int64_t* lens = pass == 0 ? dense_len : sparse_len;
+    for (int32_t i = 0; i < n; ++i) {
+      if (lens[i] < 0)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm_noalloc: negative length");
+      if (lens[i] == 0) continue;
+      if (!ptrs[i]) return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm_noalloc: null tensor");
+      if (!aligned16(ptrs[i]))
+        return fail(MOE_ERR_ALIGNMENT, "sparseclip_norm_noalloc: tensor not 16-byte aligned");
+      segs.push_back(ClipSeg{ptrs[i], lens[i], pass, 0});
+    }
+  }
+  double* partials = nullptr;
+  int32_t rc = static_partials(&partials);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t launches =
+      std::max<int64_t>(1, (static_cast<int64_t>(segs.size()) + kSegsPerLaunch - 1) / kSegsPerLaunch);
+  for (int64_t l = 0; l < launches; ++l) {
+    ClipBatch b{};
+    const size_t first = static_cast<size_t>(l) * kSegsPerLaunch;
+    b.n = static_cast<int32_t>(std::min<size_t>(kSegsPerLaunch, segs.size() - std::min(first, segs.size())));
+    for (int32_t i = 0; i < b.n; ++i) b.seg[i] = segs[first + i];
+    sumsq_kernel<<<kGrid, kBlock, 0, s>>>(b, partials + l * kGrid * 2);
+    rc = check_launch("sumsq_kernel (no-alloc)");
+    if (rc != MOE_OK) return rc;
+  }
+  finish_kernel<<<1, kBlock, 0, s>>>(partials, static_cast<int>(launches * kGrid), num_experts, out);
+  return check_launch("finish_kernel (no-alloc)");
+}
