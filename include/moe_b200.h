@@ -91,6 +91,7 @@ typedef struct moe_workspace_map {
   size_t kept_cnt;   /* [E] int32                               */
   size_t n_dropped;  /* [1] int32                               */
   size_t scratch;    /* assignment scratch (moe_assign_workspace_size bytes) */
+  size_t ffn_sync;   /* expert-FFN tile counters (moe_ffn_workspace_size bytes) */
   size_t xe;         /* [E, C, d] activations                   */
   size_t H;          /* [E, C, f] activations                   */
   size_t ye;         /* [E, C, d] activations                   */
@@ -117,6 +118,9 @@ int32_t moe_config_check(const moe_config* cfg);
 
 /* Bytes of scratch moe_topk_assign needs (0 if cfg is invalid). */
 size_t moe_assign_workspace_size(const moe_config* cfg);
+
+/* Bytes of scratch moe_expert_ffn needs (0 if cfg is invalid). */
+size_t moe_ffn_workspace_size(const moe_config* cfg);
 
 /* Layout (and total size) of the moe_layer_forward workspace. */
 int32_t moe_workspace_layout(const moe_config* cfg, moe_workspace_map* out);
@@ -168,11 +172,13 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert
  *   ye[e, r, :] = round(H[e, r, :] . W2[e]^T)          W2 [E, d, f]
  * for r < kept_cnt[e] (device int32 [E], values in 0..C).  xe, ye
  * [E, C, d] and H [E, C, f] (caller-provided scratch) in cfg->dtype; other
- * rows of H and ye are left untouched.  bf16: tcgen05 tensor cores with
- * fp32 accumulation; fp32: FMA. */
+ * rows of H and ye are left untouched.  bf16: one persistent tcgen05 kernel
+ * runs both GEMMs with fp32 accumulation; workspace holds its tile counters
+ * (moe_ffn_workspace_size bytes, zeroed by the call; unused for fp32, which
+ * runs FMA GEMMs and may pass null). */
 int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
-                       const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                       moe_stream_t stream);
+                       const int32_t* kept_cnt, void* H, void* ye, void* workspace,
+                       size_t workspace_bytes, int32_t* status, moe_stream_t stream);
 
 /* Combine (Switch notes sec. 2.1, eq. 2; drop rule sec. 2.2):
  *   y[t, :] = sum over kept j of gate[t, j] * ye[expert_idx[t, j], slot[t, j], :]
@@ -186,11 +192,14 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert
  * dispatch -> expert FFN -> combine, all on `stream`.  Wr (+ bias) for TOPK,
  * domain_id for RRE (the other may be null).  y [T, d] in cfg->dtype.
  * workspace: moe_workspace_size(cfg) bytes laid out as moe_workspace_layout
- * describes; it holds every intermediate after the call. */
+ * describes; it holds every intermediate after the call.
+ * stage_events (nullable; a profiling hook): host array of 6 cudaEvent_t
+ * (entries may be null) recorded on `stream` before the router and after
+ * the router, the assignment, the dispatch, the expert FFN and the combine. */
 int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
                           const int32_t* domain_id, const void* W1, const void* W2, void* y,
                           void* workspace, size_t workspace_bytes, int32_t* status,
-                          moe_stream_t stream);
+                          void* const* stage_events, moe_stream_t stream);
 
 /* SparseClip global gradient norm ("[Paper review] TorchScale", proposed
  * method): ||g||_2 = ||(g_d, kappa g_s)||_2 with kappa = 1/sqrt(num_experts),

@@ -40,7 +40,8 @@ class MoEConfig(ctypes.Structure):
 class WorkspaceMap(ctypes.Structure):
     """Mirror of ``moe_workspace_map``."""
     _fields_ = [(n, _sz) for n in ("logits", "expert_idx", "gate", "slot", "kept", "tok_of_row",
-                                   "arrivals", "kept_cnt", "n_dropped", "scratch", "xe", "H", "ye",
+                                   "arrivals", "kept_cnt", "n_dropped", "scratch", "ffn_sync", "xe",
+                                   "H", "ye",
                                    "total")]
 
 
@@ -61,9 +62,11 @@ SIGNATURES = {
     "moe_topk_assign": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                          _vp], _i32),
     "moe_dispatch": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
-    "moe_expert_ffn": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "moe_ffn_workspace_size": ([_PCFG], _sz),
+    "moe_expert_ffn": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp], _i32),
     "moe_combine": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
-    "moe_layer_forward": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp], _i32),
+    "moe_layer_forward": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp],
+                          _i32),
     "sparseclip_norm": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "sparseclip_norm_noalloc": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
 }
@@ -72,7 +75,7 @@ SIGNATURES = {
 def _load_library():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_fwd_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python sparse_mixture_experts_fwd_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (args, res) in SIGNATURES.items():
@@ -201,13 +204,23 @@ def dispatch(cfg, x, expert_idx, slot, kept, xe=None, stream=None):
     return xe
 
 
-def expert_ffn(cfg, xe, W1, W2, kept_cnt, H=None, ye=None, status=None, stream=None):
+def ffn_workspace_size(cfg: MoEConfig) -> int:
+    config_check(cfg)
+    return int(lib.moe_ffn_workspace_size(ctypes.byref(cfg)))
+
+
+def expert_ffn(cfg, xe, W1, W2, kept_cnt, H=None, ye=None, workspace=None, status=None,
+               stream=None):
     if H is None:
         H = torch.empty(cfg.E, cfg.capacity, cfg.d_ff, dtype=xe.dtype, device=xe.device)
     if ye is None:
         ye = torch.empty(cfg.E, cfg.capacity, cfg.d_model, dtype=xe.dtype, device=xe.device)
+    if workspace is None:
+        workspace = torch.empty(max(256, ffn_workspace_size(cfg)), dtype=torch.uint8,
+                                device=xe.device)
     _check(lib.moe_expert_ffn(ctypes.byref(cfg), _ptr(xe, "xe"), _ptr(W1, "W1"), _ptr(W2, "W2"),
                               _ptr(kept_cnt, "kept_cnt"), _ptr(H, "H"), _ptr(ye, "ye"),
+                              _ptr(workspace, "workspace"), workspace.numel(),
                               _ptr(status, "status"), _stream(stream)), "moe_expert_ffn")
     return H, ye
 
@@ -221,17 +234,34 @@ def combine(cfg, ye, expert_idx, gate, slot, kept, y=None, stream=None):
     return y
 
 
+STAGES = ("router", "route_assign", "dispatch", "expert_ffn", "combine")
+
+
 def layer_forward(cfg, x, W1, W2, *, Wr=None, bias=None, domain_id=None, y=None, workspace=None,
-                  status=None, stream=None):
-    """The whole layer on the current stream.  Returns y; ``workspace`` keeps the intermediates."""
+                  status=None, stream=None, stage_events=None):
+    """The whole layer on the current stream.  Returns y; ``workspace`` keeps the intermediates.
+
+    ``stage_events``: optional 6 ``torch.cuda.Event`` recorded before and after the
+    stages named in ``STAGES`` (a profiling hook)."""
     if y is None:
         y = torch.empty(cfg.T, cfg.d_model, dtype=x.dtype, device=x.device)
     if workspace is None:
         workspace = torch.empty(workspace_size(cfg), dtype=torch.uint8, device=x.device)
+    ev = None
+    if stage_events is not None:
+        if len(stage_events) != 6:
+            raise ValueError("stage_events needs 6 events")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        for e in stage_events:
+            if e is not None and not e.cuda_event:
+                e.record(s)  # torch creates its events lazily; the library re-records them
+        ev = (ctypes.c_void_p * 6)(*[e.cuda_event if e is not None else None for e in stage_events])
     _check(lib.moe_layer_forward(ctypes.byref(cfg), _ptr(x, "x"), _ptr(Wr, "Wr"), _ptr(bias, "bias"),
                                  _ptr(domain_id, "domain_id"), _ptr(W1, "W1"), _ptr(W2, "W2"),
                                  _ptr(y, "y"), _ptr(workspace, "workspace"), workspace.numel(),
-                                 _ptr(status, "status"), _stream(stream)), "moe_layer_forward")
+                                 _ptr(status, "status"),
+                                 None if ev is None else ctypes.cast(ev, _vp), _stream(stream)),
+           "moe_layer_forward")
     return y
 
 

@@ -4,7 +4,8 @@ Each ``csrc/*.cu`` file is compiled by nvcc (in parallel) into
 ``_build/*.o`` and linked into ``sparse_mixture_experts_fwd_b200/libmoe_b200.so``
 with the CUDA runtime linked statically, so the library loads on a machine
 without a GPU driver (the driver is reached at run time through the runtime).
-``python -m sparse_mixture_experts_fwd_b200.build`` rebuilds what changed;
+``python sparse_mixture_experts_fwd_b200/build.py`` rebuilds what changed (run it
+by path: importing the package itself needs the built library);
 ``--ptxas-info`` also writes ptxas register/spill reports to ``_build/``.
 """
 from __future__ import annotations

@@ -119,6 +119,7 @@ void layout(const moe_config& c, moe_workspace_map* m) {
   m->kept_cnt = take(E * 4);
   m->n_dropped = take(4);
   m->scratch = take(assign_scratch_bytes(c));
+  m->ffn_sync = take(ffn_sync_bytes(c));
   m->xe = take(E * C * static_cast<size_t>(c.d_model) * es);
   m->H = take(E * C * static_cast<size_t>(c.d_ff) * es);
   m->ye = take(E * C * static_cast<size_t>(c.d_model) * es);
@@ -237,9 +238,14 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert
   return launch_dispatch(*cfg, x, expert_idx, slot, kept, xe, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t moe_ffn_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return ffn_sync_bytes(*cfg);
+}
+
 int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
-                       const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                       moe_stream_t stream) {
+                       const int32_t* kept_cnt, void* H, void* ye, void* workspace,
+                       size_t workspace_bytes, int32_t* status, moe_stream_t stream) {
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   if (cfg->capacity == 0) return MOE_OK;
@@ -250,7 +256,13 @@ int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, co
   MOE_TRY(need_ptr(H, "H"));
   MOE_TRY(need_ptr(ye, "ye"));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cfg->dtype == MOE_DTYPE_BF16) return launch_ffn_tc(*cfg, xe, W1, W2, kept_cnt, H, ye, status, s);
+  if (cfg->dtype == MOE_DTYPE_BF16) {
+    const size_t need = ffn_sync_bytes(*cfg);
+    if (!workspace || workspace_bytes < need)
+      return fail(MOE_ERR_WORKSPACE, "moe_expert_ffn: workspace needs " + std::to_string(need) + " bytes");
+    MOE_TRY(need_ptr(workspace, "workspace"));
+    return launch_ffn_tc(*cfg, xe, W1, W2, kept_cnt, H, ye, workspace, false, status, s);
+  }
   return launch_ffn_f32(*cfg, xe, W1, W2, kept_cnt, H, ye, s);
 }
 
@@ -272,7 +284,7 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert
 int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
                           const int32_t* domain_id, const void* W1, const void* W2, void* y,
                           void* workspace, size_t workspace_bytes, int32_t* status,
-                          moe_stream_t stream) {
+                          void* const* stage_events, moe_stream_t stream) {
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   const moe_config& c = *cfg;
@@ -311,16 +323,35 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
   void* H = ws + m.H;
   void* ye = ws + m.ye;
 
+  auto mark = [&](int i) -> int32_t {
+    if (!stage_events || !stage_events[i]) return MOE_OK;
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s);
+    return e == cudaSuccess ? MOE_OK
+                            : fail(MOE_ERR_CUDA, std::string("cudaEventRecord: ") + cudaGetErrorString(e));
+  };
+  // the fused expert FFN's counters are cleared by the dispatch kernel
+  unsigned int* ffn_sync = reinterpret_cast<unsigned int*>(ws + m.ffn_sync);
+  const bool dispatch_zeroes = c.T > 0 && c.capacity > 0 && c.dtype == MOE_DTYPE_BF16;
+  const int n_sync_words = static_cast<int>(ffn_sync_bytes(c) / sizeof(unsigned int));
+
+  MOE_TRY(mark(0));
   if (c.mode == MOE_ROUTE_TOPK && c.T > 0) {
     if (c.dtype == MOE_DTYPE_BF16) MOE_TRY(launch_router_tc(c, x, Wr, bias, logits, status, s));
     else MOE_TRY(launch_router_f32(c, x, Wr, bias, logits, s));
   }
+  MOE_TRY(mark(1));
   MOE_TRY(launch_route_assign(c, logits, domain_id, expert_idx, gate, slot, kept, tok_of_row,
                               arrivals, kept_cnt, n_dropped, scratch, status, s));
-  MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, s));
-  if (c.dtype == MOE_DTYPE_BF16) MOE_TRY(launch_ffn_tc(c, xe, W1, W2, kept_cnt, H, ye, status, s));
+  MOE_TRY(mark(2));
+  MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, s,
+                          dispatch_zeroes ? ffn_sync : nullptr, dispatch_zeroes ? n_sync_words : 0));
+  MOE_TRY(mark(3));
+  if (c.dtype == MOE_DTYPE_BF16)
+    MOE_TRY(launch_ffn_tc(c, xe, W1, W2, kept_cnt, H, ye, ffn_sync, dispatch_zeroes, status, s));
   else MOE_TRY(launch_ffn_f32(c, xe, W1, W2, kept_cnt, H, ye, s));
-  return launch_combine(c, ye, expert_idx, gate, slot, kept, y, s);
+  MOE_TRY(mark(4));
+  MOE_TRY(launch_combine(c, ye, expert_idx, gate, slot, kept, y, s));
+  return mark(5);
 }
 
 }  // extern "C"

@@ -5,9 +5,8 @@
 // for every group g (an expert, or the single router group), m < rows[g]
 // (read on the device, e.g. the kept-token count of an expert) and n < N.
 // Both operands are K-major bf16; accumulation is fp32 in tensor memory.
-// It serves the two dense contractions of the layer:
-//   * expert FFN (Switch notes sec. 2.1, E_i): H = ReLU(xe W1^T), ye = H W2^T
-//   * router logits (sec. 2.1 h = W_r x, fp32 per sec. 2.4): x Wr^T + bias
+// It computes the router logits (Switch notes sec. 2.1 h = W_r x, fp32 per
+// sec. 2.4): x Wr^T + bias.  (The expert FFN has its own fused kernel.)
 //
 // Design: one persistent CTA per SM walks a static list of 128 x BN output
 // tiles ordered (group, n-block, m-block) so that the m-blocks sharing a
@@ -364,10 +363,12 @@ int32_t launch_gemm(const void* A, uint64_t a_rows, const void* B, uint64_t b_ro
 
 }  // namespace
 
-// H = ReLU(xe W1^T), ye = H W2^T over each expert's kept rows.
-int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const void* W2,
-                      const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                      cudaStream_t s) {
+// Expert FFN as two grouped launches (GEMM 1 then GEMM 2), used when experts
+// span several 128-row blocks: the static tile order keeps the CTAs that
+// share a weight tile in lockstep, so its k-slices are served once from L2.
+int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1, const void* W2,
+                            const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
+                            cudaStream_t s) {
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
   const int64_t mblk_max = (C + kBM - 1) / kBM;

@@ -32,9 +32,15 @@ int32_t launch_router_tc(const moe_config& c, const void* x, const void* Wr, con
                          float* logits, int32_t* status, cudaStream_t s);
 int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, const float* bias,
                           float* logits, cudaStream_t s);
+int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1, const void* W2,
+                            const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
+                            cudaStream_t s);
+// sync: ffn_sync_bytes(c) bytes of scratch; sync_zeroed says the caller
+// already zeroed it on this stream (else the launcher does).
+size_t ffn_sync_bytes(const moe_config& c);
 int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const void* W2,
-                      const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                      cudaStream_t s);
+                      const int32_t* kept_cnt, void* H, void* ye, void* sync, bool sync_zeroed,
+                      int32_t* status, cudaStream_t s);
 int32_t launch_ffn_f32(const moe_config& c, const void* xe, const void* W1, const void* W2,
                        const int32_t* kept_cnt, void* H, void* ye, cudaStream_t s);
 int32_t launch_route_assign(const moe_config& c, const float* logits, const int32_t* domain,
@@ -43,8 +49,10 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
                             int32_t* n_dropped, void* scratch, int32_t* status,
                             cudaStream_t s);
 size_t assign_scratch_bytes(const moe_config& c);
+// zero_words (nullable): n_zero words the dispatch kernel clears for the next kernel
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
-                        const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s);
+                        const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
+                        unsigned int* zero_words = nullptr, int n_zero = 0);
 int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* expert_idx,
                        const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
                        cudaStream_t s);

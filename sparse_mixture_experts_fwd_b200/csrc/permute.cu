@@ -22,9 +22,14 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
                                                        const int32_t* __restrict__ expert_idx,
                                                        const int32_t* __restrict__ slot,
                                                        const uint8_t* __restrict__ kept,
-                                                       uint4* __restrict__ xe) {
+                                                       uint4* __restrict__ xe,
+                                                       unsigned int* __restrict__ zero_words,
+                                                       int n_zero) {
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  // counters the next kernel on this stream expects at zero (the fused expert FFN)
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0u;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
        t += nwarps) {
     int64_t dst[K];
@@ -139,16 +144,19 @@ unsigned grid_for_tokens(int64_t T) {
 }  // namespace
 
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
-                        const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s) {
+                        const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
+                        unsigned int* zero_words, int n_zero) {
   if (c.T == 0 || c.capacity == 0) return MOE_OK;
   const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
   const unsigned grid = grid_for_tokens(c.T);
   if (c.k == 1)
     dispatch_kernel<1><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
-                                            expert_idx, slot, kept, static_cast<uint4*>(xe));
+                                            expert_idx, slot, kept, static_cast<uint4*>(xe),
+                                            zero_words, n_zero);
   else
     dispatch_kernel<2><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
-                                            expert_idx, slot, kept, static_cast<uint4*>(xe));
+                                            expert_idx, slot, kept, static_cast<uint4*>(xe),
+                                            zero_words, n_zero);
   return check_launch("dispatch_kernel");
 }
 

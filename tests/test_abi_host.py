@@ -83,7 +83,7 @@ def test_config_accepts_workloads(moe):
         m = moe.workspace_layout(c)
         es = 2 if w.dtype == "bf16" else 4
         offs = [m.logits, m.expert_idx, m.gate, m.slot, m.kept, m.tok_of_row, m.arrivals,
-                m.kept_cnt, m.n_dropped, m.scratch, m.xe, m.H, m.ye, m.total]
+                m.kept_cnt, m.n_dropped, m.scratch, m.ffn_sync, m.xe, m.H, m.ye, m.total]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert m.total - m.ye >= w.E * C * w.d_model * es
         assert m.ye - m.H >= w.E * C * w.d_ff * es
@@ -98,13 +98,17 @@ def test_calls_rejected_on_host(moe):
     # misaligned logits
     assert moe.lib.moe_router(ctypes.byref(c), p, p, None, ctypes.c_void_p(4100), None, None) == -3
     # workspace too small
-    assert moe.lib.moe_layer_forward(ctypes.byref(c), p, p, None, None, p, p, p, p, 10, None, None) == -4
+    assert moe.lib.moe_layer_forward(ctypes.byref(c), p, p, None, None, p, p, p, p, 10, None, None,
+                                     None) == -4
     # topk_assign without workspace
     assert moe.lib.moe_topk_assign(ctypes.byref(c), p, None, p, p, p, p, p, p, p, p, None, 0,
                                    None, None) == -4
     # invalid config reaches no launch
     bad = cfg(moe, k=3)
-    assert moe.lib.moe_expert_ffn(ctypes.byref(bad), p, p, p, p, p, p, None, None) == -2
+    assert moe.lib.moe_expert_ffn(ctypes.byref(bad), p, p, p, p, p, p, p, 4096, None, None) == -2
+    # bf16 expert FFN without its tile-counter workspace
+    assert moe.lib.moe_expert_ffn(ctypes.byref(c), p, p, p, p, p, p, None, 0, None, None) == -4
+    assert moe.lib.moe_ffn_workspace_size(ctypes.byref(c)) == 768  # 4 * (1 + 128) -> 256-aligned
     assert moe.lib.moe_dispatch(None, p, p, p, p, p, None) == -1
     # sparseclip
     assert moe.lib.sparseclip_norm(None, None, 0, None, None, 0, 0, p, p, 1 << 20, None) == -1

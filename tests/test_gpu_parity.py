@@ -193,12 +193,21 @@ def test_combine(moe, cuda_device, case):
 # a6 expert FFN
 # ---------------------------------------------------------------------------
 
+FFN_SHAPES = {
+    # C > 128: the two-launch grouped GEMM
+    "multi_block": (5, 300, 256, 768, [300, 0, 129, 1, 128]),
+    # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
+    "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
+}
+
+
+@pytest.mark.parametrize("shape", sorted(FFN_SHAPES))
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_expert_ffn_ragged_tiles(moe, cuda_device, dtype):
+def test_expert_ffn_ragged_tiles(moe, cuda_device, dtype, shape):
     """Several 128-row and 256-column tiles, ragged kept counts, C not a tile multiple."""
     dev = cuda_device
-    E, C, d, f = 5, 300, 256, 768
-    kept = torch.tensor([300, 0, 129, 1, 128], dtype=torch.int32)
+    E, C, d, f, kept_list = FFN_SHAPES[shape]
+    kept = torch.tensor(kept_list, dtype=torch.int32)
     xe = synth.normal(21, 1, (E, C, d), 1.0, dtype)
     W1 = synth.normal(21, 3, (E, f, d), 0.02, dtype)
     W2 = synth.normal(21, 4, (E, d, f), 0.02, dtype)
@@ -309,7 +318,11 @@ def test_layer_forward_deterministic(moe, cuda_device, case):
     D = case.dev
     kw = dict(Wr=D["Wr"], bias=D["bias"], domain_id=D["domain"])
     y1 = moe.layer_forward(case.cfg, D["x"], D["W1"], D["W2"], **kw)
-    y2 = moe.layer_forward(case.cfg, D["x"], D["W1"], D["W2"], **kw)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    y2 = moe.layer_forward(case.cfg, D["x"], D["W1"], D["W2"], stage_events=evs, **kw)
+    torch.cuda.synchronize()
+    stage_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(5)]  # the profiling hook
+    assert all(t >= 0 for t in stage_ms) and evs[0].elapsed_time(evs[5]) > 0
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int32 if case.w.dtype == "f32" else torch.int16),
                        y2.view(torch.int32 if case.w.dtype == "f32" else torch.int16))
