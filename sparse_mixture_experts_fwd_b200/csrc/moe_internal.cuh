@@ -49,6 +49,9 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
                             int32_t* n_dropped, void* scratch, int32_t* status,
                             cudaStream_t s);
 size_t assign_scratch_bytes(const moe_config& c);
+int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* slot,
+                      uint8_t* kept, int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
+                      int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s);
 // zero_words (nullable): n_zero words the dispatch kernel clears for the next kernel
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
                         const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,

@@ -7,18 +7,21 @@
 // the same way with the first excluded, and the softmax denominator
 // sum_j exp(h_j - max) with a shuffle sum; gate = exp(h_i - max) / sum.
 //
-// Slot assignment (sec. 2.2, eq. 3 and the drop rule), in token order:
-//   rank kernel     each 1024-assignment block ranks its choices per expert:
-//                   __match_any_sync groups the lanes that chose the same
-//                   expert, __popc of the lower peers gives the rank inside
-//                   the warp, and per-warp counts are prefix-summed in shared
-//                   memory across the 32 warps; block totals go to a
-//                   [blocks, E] histogram;
-//   scan kernel     one thread per expert turns the histogram into exclusive
-//                   block offsets and yields arrivals, kept counts and the
-//                   dropped total;
-//   finalize kernel slot = block offset + rank, kept = slot < C, and the
-//                   [E, C] row -> token map.
+// Slot assignment (sec. 2.2, eq. 3 and the drop rule), in token order, as ONE
+// kernel over blocks of 1024 choices (choice a = t*k + j):
+//   1. rank inside the block: __match_any_sync groups the lanes that chose
+//      the same expert, __popc of the lower peers gives the rank inside the
+//      warp, per-warp counts are prefix-summed in shared memory across the 32
+//      warps; the block's per-expert counts are its aggregate;
+//   2. decoupled look-back: the block publishes its aggregate (flag 1), reads
+//      the flags of all earlier blocks, and sums their aggregates back to the
+//      nearest block that already published its inclusive prefix (flag 2),
+//      then publishes its own inclusive prefix (flag 2);
+//   3. slot = exclusive prefix + rank, kept = slot < C, row -> token map;
+//      the last block also writes arrivals, kept counts, the dropped total
+//      and marks free rows of the map with -1.
+// The flags are cleared by the kernel that produced the choices (stream
+// order), and every wait on a flag is bounded by time.
 #include <climits>
 #include <cmath>
 
@@ -35,6 +38,11 @@ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t t) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
   return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ void clear_flags(unsigned int* flags, int nblk) {
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nblk; i += blockDim.x) flags[i] = 0u;
 }
 
 // logits[t, e] = sum_c x[t, c] * Wr[e, c] + bias[e]   (fp32 FMA chain in c order)
@@ -70,7 +78,9 @@ template <int K>
 __global__ void __launch_bounds__(256) gate_topk_kernel(int64_t T, int E,
                                                         const float* __restrict__ logits,
                                                         int32_t* __restrict__ expert_idx,
-                                                        float* __restrict__ gate) {
+                                                        float* __restrict__ gate,
+                                                        unsigned int* flags, int nblk) {
+  clear_flags(flags, nblk);
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
@@ -123,7 +133,8 @@ __global__ void __launch_bounds__(256) gate_topk_kernel(int64_t T, int E,
 __global__ void route_rre_kernel(int64_t T, int E, int G, uint64_t seed,
                                  const int32_t* __restrict__ domain,
                                  int32_t* __restrict__ expert_idx, float* __restrict__ gate,
-                                 int32_t* status) {
+                                 int32_t* status, unsigned int* flags, int nblk) {
+  clear_flags(flags, nblk);
   const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (t >= T) return;
   const int per = E / G;
@@ -137,19 +148,47 @@ __global__ void route_rre_kernel(int64_t T, int E, int G, uint64_t seed,
   gate[t] = 1.0f;
 }
 
-// rank of each choice among the same expert's choices inside its 1024-block
-__global__ void __launch_bounds__(kAssignBlock) assign_rank_kernel(
-    int64_t n_assign, int E, const int32_t* __restrict__ expert_idx, int32_t* __restrict__ rank,
-    int32_t* __restrict__ block_hist) {
-  extern __shared__ int s_cnt[];  // [32 warps][E]
+MOE_DEV unsigned int ld_acquire(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+MOE_DEV void st_release(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+struct AssignArgs {
+  int64_t n_assign;
+  int k, E, C, nblk;
+  const int32_t* expert_idx;
+  int32_t* slot;
+  uint8_t* kept;
+  int32_t* tok_of_row;
+  int32_t* arrivals;
+  int32_t* kept_cnt;
+  int32_t* n_dropped;
+  unsigned int* flags;  // [nblk], cleared before launch
+  int32_t* aggr;        // [nblk][E]
+  int32_t* incl;        // [nblk][E]
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArgs p) {
+  extern __shared__ int s_cnt[];  // [32 warps][E], then excl[E]
+  __shared__ int s_pstar, s_ok, s_maxinc, s_maxbad, s_drop[32];
+  int* s_excl = s_cnt + 32 * p.E;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.x;
+  const int E = p.E;
+
+  // 1. ranks inside the block
   for (int i = tid; i < 32 * E; i += kAssignBlock) s_cnt[i] = 0;
   __syncthreads();
-  const int64_t a = static_cast<int64_t>(blockIdx.x) * kAssignBlock + tid;
-  int e = a < n_assign ? __ldg(expert_idx + a) : -1;
+  const int64_t a = static_cast<int64_t>(b) * kAssignBlock + tid;
+  int e = a < p.n_assign ? __ldg(p.expert_idx + a) : -1;
   if (e >= E) e = -1;
   const unsigned peers = __match_any_sync(0xffffffffu, e);
-  const int r = __popc(peers & ((1u << lane) - 1u));
+  const int r_in_warp = __popc(peers & ((1u << lane) - 1u));
   if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * E + e] = __popc(peers);
   __syncthreads();
   for (int x = tid; x < E; x += kAssignBlock) {
@@ -159,72 +198,119 @@ __global__ void __launch_bounds__(kAssignBlock) assign_rank_kernel(
       s_cnt[w * E + x] = run;
       run += c;
     }
-    block_hist[static_cast<int64_t>(blockIdx.x) * E + x] = run;
+    p.aggr[static_cast<int64_t>(b) * E + x] = run;  // block aggregate
+    s_excl[x] = 0;
+    if (b == 0) p.incl[x] = run;
   }
+  // 2. publish the aggregate (or, for block 0, the inclusive prefix)
+  __threadfence();
   __syncthreads();
-  if (e >= 0) rank[a] = s_cnt[warp * E + e] + r;
-}
+  if (tid == 0) st_release(p.flags + b, b == 0 ? 2u : 1u);
 
-// per expert: exclusive scan of the block histogram -> block offsets, arrivals, kept, dropped
-__global__ void __launch_bounds__(256) assign_scan_kernel(int nblk, int E, int C,
-                                                          int32_t* __restrict__ block_hist,
-                                                          int32_t* __restrict__ arrivals,
-                                                          int32_t* __restrict__ kept_cnt,
-                                                          int32_t* __restrict__ n_dropped) {
-  __shared__ int s_drop[256];
-  int drop = 0;
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int c = block_hist[static_cast<int64_t>(b) * E + x];
-      block_hist[static_cast<int64_t>(b) * E + x] = run;
-      run += c;
+  if (b > 0) {
+    // p*: the latest earlier block with an inclusive prefix, usable once every
+    // block after it has at least published its aggregate.  All earlier flags
+    // are read in parallel (one thread each) and reduced in shared memory.
+    const unsigned long long t0 = dev::globaltimer();
+    for (;;) {
+      if (tid == 0) {
+        s_maxinc = -1;
+        s_maxbad = -1;
+      }
+      __syncthreads();
+      for (int q = tid; q < b; q += kAssignBlock) {
+        const unsigned int f = ld_acquire(p.flags + q);
+        if (f == 2u) atomicMax(&s_maxinc, q);
+        else if (f == 0u) atomicMax(&s_maxbad, q);
+      }
+      __syncthreads();
+      const bool ready = s_maxinc >= 0 && s_maxbad < s_maxinc;
+      if (tid == 0) {
+        s_pstar = s_maxinc;
+        s_ok = ready ? 1 : (dev::globaltimer() - t0 > dev::kWaitLimitNs ? -1 : 0);
+        if (s_ok < 0 && p.status) atomicOr(p.status, MOE_STATUS_TIMEOUT);
+      }
+      __syncthreads();
+      if (s_ok != 0) break;
     }
-    arrivals[x] = run;
-    kept_cnt[x] = run < C ? run : C;
-    drop += run > C ? run - C : 0;
-  }
-  s_drop[threadIdx.x] = drop;
-  __syncthreads();
-  for (int off = 128; off > 0; off >>= 1) {
-    if (threadIdx.x < off) s_drop[threadIdx.x] += s_drop[threadIdx.x + off];
+    if (s_ok < 0) return;  // bounded wait expired: outputs are invalid, status says so
+    const int pstar = s_pstar;
+    for (int x = tid; x < E; x += kAssignBlock) {
+      int acc = __ldcg(p.incl + static_cast<int64_t>(pstar) * E + x);
+      for (int q = pstar + 1; q < b; ++q) acc += __ldcg(p.aggr + static_cast<int64_t>(q) * E + x);
+      s_excl[x] = acc;
+      p.incl[static_cast<int64_t>(b) * E + x] = acc + p.aggr[static_cast<int64_t>(b) * E + x];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release(p.flags + b, 2u);
+  } else {
     __syncthreads();
   }
-  if (threadIdx.x == 0) n_dropped[0] = s_drop[0];
-}
 
-__global__ void __launch_bounds__(256) assign_finalize_kernel(
-    int64_t n_assign, int k, int E, int C, const int32_t* __restrict__ expert_idx,
-    const int32_t* __restrict__ block_off, int32_t* __restrict__ slot, uint8_t* __restrict__ kept,
-    int32_t* __restrict__ tok_of_row, const int32_t* __restrict__ kept_cnt) {
-  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (i < n_assign) {
-    const int e = expert_idx[i];
-    if (e >= 0 && e < E) {
-      const int s = block_off[(i / kAssignBlock) * E + e] + slot[i];
-      slot[i] = s;
-      const bool kp = s < C;
-      kept[i] = kp ? 1 : 0;
-      if (kp) tok_of_row[static_cast<int64_t>(e) * C + s] = static_cast<int32_t>(i / k);
+  // 3. slots, kept mask, row -> token map
+  if (a < p.n_assign) {
+    if (e >= 0) {
+      const int s = s_excl[e] + s_cnt[warp * E + e] + r_in_warp;
+      p.slot[a] = s;
+      const bool kp = s < p.C;
+      p.kept[a] = kp ? 1 : 0;
+      if (kp) p.tok_of_row[static_cast<int64_t>(e) * p.C + s] = static_cast<int32_t>(a / p.k);
     } else {
-      slot[i] = INT_MAX;
-      kept[i] = 0;
+      p.slot[a] = INT_MAX;
+      p.kept[a] = 0;
     }
   }
-  if (C > 0 && i < static_cast<int64_t>(E) * C) {
-    const int e = static_cast<int>(i / C);
-    const int r = static_cast<int>(i - static_cast<int64_t>(e) * C);
-    if (r >= kept_cnt[e]) tok_of_row[i] = -1;
+  // the last block owns the totals
+  if (b == p.nblk - 1) {
+    __syncthreads();  // every thread is done reading the rank table reused below
+    int drop = 0;
+    for (int x = tid; x < E; x += kAssignBlock) {
+      const int arr = s_excl[x] + p.aggr[static_cast<int64_t>(b) * E + x];
+      p.arrivals[x] = arr;
+      const int kc = arr < p.C ? arr : p.C;
+      p.kept_cnt[x] = kc;
+      s_cnt[x] = kc;  // reuse: kept count per expert for the -1 fill below
+      drop += arr - kc;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) drop += __shfl_xor_sync(0xffffffffu, drop, off);
+    if (lane == 0) s_drop[warp] = drop;
+    __syncthreads();
+    if (tid == 0) {
+      int tot = 0;
+      for (int w = 0; w < 32; ++w) tot += s_drop[w];
+      p.n_dropped[0] = tot;
+    }
+    const int64_t rows = static_cast<int64_t>(E) * p.C;
+    for (int64_t i = tid; i < rows; i += kAssignBlock) {
+      const int ex = static_cast<int>(i / p.C);
+      if (static_cast<int>(i - static_cast<int64_t>(ex) * p.C) >= s_cnt[ex]) p.tok_of_row[i] = -1;
+    }
   }
+}
+
+// Totals for a call with no choices (T = 0): zero counts, empty row map.
+__global__ void assign_empty_kernel(int E, int C, int32_t* arrivals, int32_t* kept_cnt,
+                                    int32_t* n_dropped, int32_t* tok_of_row) {
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    arrivals[x] = 0;
+    kept_cnt[x] = 0;
+  }
+  if (threadIdx.x == 0) n_dropped[0] = 0;
+  const int64_t rows = static_cast<int64_t>(E) * C;
+  for (int64_t i = threadIdx.x; i < rows; i += blockDim.x) tok_of_row[i] = -1;
 }
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace
 
+// flags [nblk] u32, then aggr and incl [nblk][E] i32 each
 size_t assign_scratch_bytes(const moe_config& c) {
-  const int64_t n_assign = c.T * c.k;
-  return align256(static_cast<size_t>(ceil_div(n_assign, kAssignBlock)) * c.E * sizeof(int32_t));
+  const int64_t nblk = ceil_div(c.T * c.k, kAssignBlock);
+  return align256(static_cast<size_t>(nblk) * sizeof(unsigned int)) +
+         2 * align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
 }
 
 int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, const float* bias,
@@ -243,43 +329,74 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
                             int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s) {
   const int64_t T = c.T;
   const int64_t n_assign = T * c.k;
-  if (T > 0) {
-    if (c.mode == MOE_ROUTE_TOPK) {
-      const int64_t blocks = std::min<int64_t>(ceil_div(T, 8), int64_t(num_sms()) * 16);
-      if (c.k == 1)
-        gate_topk_kernel<1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(T, c.E, logits,
-                                                                          expert_idx, gate);
-      else
-        gate_topk_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(T, c.E, logits,
-                                                                          expert_idx, gate);
-      int32_t rc = check_launch("gate_topk_kernel");
-      if (rc != MOE_OK) return rc;
-    } else {
-      route_rre_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, s>>>(
-          T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status);
-      int32_t rc = check_launch("route_rre_kernel");
-      if (rc != MOE_OK) return rc;
-    }
-  }
-  int32_t* block_hist = static_cast<int32_t*>(scratch);
   const int64_t nblk = ceil_div(n_assign, kAssignBlock);
-  if (nblk > 0) {
-    assign_rank_kernel<<<static_cast<unsigned>(nblk), kAssignBlock, 32 * c.E * sizeof(int), s>>>(
-        n_assign, c.E, expert_idx, slot, block_hist);
-    int32_t rc = check_launch("assign_rank_kernel");
+  char* sc = static_cast<char*>(scratch);
+  unsigned int* flags = reinterpret_cast<unsigned int*>(sc);
+  const size_t flags_bytes = align256(static_cast<size_t>(nblk) * sizeof(unsigned int));
+  const size_t vec_bytes = align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
+  int32_t* aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
+  int32_t* incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
+  if (T == 0) {
+    assign_empty_kernel<<<1, 256, 0, s>>>(c.E, c.capacity, arrivals, kept_cnt, n_dropped,
+                                          tok_of_row);
+    return check_launch("assign_empty_kernel");
+  }
+  if (c.mode == MOE_ROUTE_TOPK) {
+    const int64_t blocks = std::min<int64_t>(ceil_div(T, 8), int64_t(num_sms()) * 16);
+    if (c.k == 1)
+      gate_topk_kernel<1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+          T, c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
+    else
+      gate_topk_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+          T, c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
+    int32_t rc = check_launch("gate_topk_kernel");
+    if (rc != MOE_OK) return rc;
+  } else {
+    route_rre_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, s>>>(
+        T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status, flags,
+        static_cast<int>(nblk));
+    int32_t rc = check_launch("route_rre_kernel");
     if (rc != MOE_OK) return rc;
   }
-  assign_scan_kernel<<<1, 256, 0, s>>>(static_cast<int>(nblk), c.E, c.capacity, block_hist,
-                                       arrivals, kept_cnt, n_dropped);
-  int32_t rc = check_launch("assign_scan_kernel");
-  if (rc != MOE_OK) return rc;
-  const int64_t n_fin = std::max<int64_t>(n_assign, int64_t(c.E) * c.capacity);
-  if (n_fin > 0) {
-    assign_finalize_kernel<<<static_cast<unsigned>(ceil_div(n_fin, 256)), 256, 0, s>>>(
-        n_assign, c.k, c.E, c.capacity, expert_idx, block_hist, slot, kept, tok_of_row, kept_cnt);
-    rc = check_launch("assign_finalize_kernel");
+  return launch_assign(c, expert_idx, slot, kept, tok_of_row, arrivals, kept_cnt, n_dropped,
+                       scratch, status, s);
+}
+
+// The slot assignment alone, from choices whose look-back flags are already
+// cleared (by the kernel that produced them, earlier on the same stream).
+int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* slot,
+                      uint8_t* kept, int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
+                      int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s) {
+  const int64_t n_assign = c.T * c.k;
+  const int64_t nblk = ceil_div(n_assign, kAssignBlock);
+  if (nblk == 0) {
+    assign_empty_kernel<<<1, 256, 0, s>>>(c.E, c.capacity, arrivals, kept_cnt, n_dropped,
+                                          tok_of_row);
+    return check_launch("assign_empty_kernel");
   }
-  return rc;
+  char* sc = static_cast<char*>(scratch);
+  const size_t flags_bytes = align256(static_cast<size_t>(nblk) * sizeof(unsigned int));
+  const size_t vec_bytes = align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
+  AssignArgs p{};
+  p.n_assign = n_assign;
+  p.k = c.k;
+  p.E = c.E;
+  p.C = c.capacity;
+  p.nblk = static_cast<int>(nblk);
+  p.expert_idx = expert_idx;
+  p.slot = slot;
+  p.kept = kept;
+  p.tok_of_row = tok_of_row;
+  p.arrivals = arrivals;
+  p.kept_cnt = kept_cnt;
+  p.n_dropped = n_dropped;
+  p.flags = reinterpret_cast<unsigned int*>(sc);
+  p.aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
+  p.incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
+  p.status = status;
+  const size_t smem = (33 * static_cast<size_t>(c.E)) * sizeof(int);
+  assign_kernel<<<static_cast<unsigned>(nblk), kAssignBlock, smem, s>>>(p);
+  return check_launch("assign_kernel");
 }
 
 }  // namespace moe
