@@ -81,7 +81,9 @@ typedef struct moe_config {
  * workspace base (each 256-byte aligned) and the total size.  After a call
  * the caller may read any of these intermediate tensors. */
 typedef struct moe_workspace_map {
-  size_t logits;     /* [T, E] fp32 (TOPK only)                 */
+  size_t logits;     /* [T, E] fp32 (fp32 TOPK layers only; bf16
+                        layers fuse the gate into the router and
+                        keep no logits: the region is empty)   */
   size_t expert_idx; /* [T, k] int32                            */
   size_t gate;       /* [T, k] fp32                             */
   size_t slot;       /* [T, k] int32                            */

@@ -288,7 +288,7 @@ def workspace_views(cfg, workspace) -> dict:
         H=view(m.H, E * C * f, act, (E, C, f), es),
         ye=view(m.ye, E * C * d, act, (E, C, d), es),
     )
-    if cfg.mode == ROUTE_TOPK:
+    if cfg.mode == ROUTE_TOPK and cfg.dtype == DTYPE_F32:  # bf16 layers keep no logits
         v["logits"] = view(m.logits, T * E, torch.float32, (T, E), 4)
     return v
 

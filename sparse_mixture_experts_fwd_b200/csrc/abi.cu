@@ -109,7 +109,8 @@ void layout(const moe_config& c, moe_workspace_map* m) {
     off += align256(bytes);
     return o;
   };
-  m->logits = take(c.mode == MOE_ROUTE_TOPK ? T * E * 4 : 0);
+  // bf16 layers fuse the gate into the router, so only fp32 top-k layers keep logits
+  m->logits = take(c.mode == MOE_ROUTE_TOPK && c.dtype == MOE_DTYPE_F32 ? T * E * 4 : 0);
   m->expert_idx = take(T * k * 4);
   m->gate = take(T * k * 4);
   m->slot = take(T * k * 4);
@@ -335,13 +336,22 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
   const int n_sync_words = static_cast<int>(ffn_sync_bytes(c) / sizeof(unsigned int));
 
   MOE_TRY(mark(0));
-  if (c.mode == MOE_ROUTE_TOPK && c.T > 0) {
-    if (c.dtype == MOE_DTYPE_BF16) MOE_TRY(launch_router_tc(c, x, Wr, bias, logits, status, s));
-    else MOE_TRY(launch_router_f32(c, x, Wr, bias, logits, s));
+  const bool fused_router = c.mode == MOE_ROUTE_TOPK && c.dtype == MOE_DTYPE_BF16 && c.T > 0;
+  if (fused_router) {
+    // router GEMM with the gate and top-k in its epilogue (no logits round trip)
+    MOE_TRY(launch_router_topk_tc(c, x, Wr, bias, expert_idx, gate,
+                                  static_cast<unsigned int*>(scratch), assign_flag_words(c),
+                                  status, s));
+  } else if (c.mode == MOE_ROUTE_TOPK && c.T > 0) {
+    MOE_TRY(launch_router_f32(c, x, Wr, bias, logits, s));
   }
   MOE_TRY(mark(1));
-  MOE_TRY(launch_route_assign(c, logits, domain_id, expert_idx, gate, slot, kept, tok_of_row,
-                              arrivals, kept_cnt, n_dropped, scratch, status, s));
+  if (fused_router)
+    MOE_TRY(launch_assign(c, expert_idx, slot, kept, tok_of_row, arrivals, kept_cnt, n_dropped,
+                          scratch, status, s));
+  else
+    MOE_TRY(launch_route_assign(c, logits, domain_id, expert_idx, gate, slot, kept, tok_of_row,
+                                arrivals, kept_cnt, n_dropped, scratch, status, s));
   MOE_TRY(mark(2));
   MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, s,
                           dispatch_zeroes ? ffn_sync : nullptr, dispatch_zeroes ? n_sync_words : 0));

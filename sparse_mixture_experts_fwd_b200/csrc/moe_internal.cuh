@@ -49,6 +49,12 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
                             int32_t* n_dropped, void* scratch, int32_t* status,
                             cudaStream_t s);
 size_t assign_scratch_bytes(const moe_config& c);
+// look-back flags at the start of the assignment scratch; the kernel that
+// produces the choices zeroes them
+int assign_flag_words(const moe_config& c);
+int32_t launch_router_topk_tc(const moe_config& c, const void* x, const void* Wr,
+                              const float* bias, int32_t* expert_idx, float* gate,
+                              unsigned int* clear, int n_clear, int32_t* status, cudaStream_t s);
 int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* slot,
                       uint8_t* kept, int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
                       int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s);

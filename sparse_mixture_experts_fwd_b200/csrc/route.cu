@@ -306,6 +306,10 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace
 
+int assign_flag_words(const moe_config& c) {
+  return static_cast<int>(ceil_div(c.T * c.k, kAssignBlock));
+}
+
 // flags [nblk] u32, then aggr and incl [nblk][E] i32 each
 size_t assign_scratch_bytes(const moe_config& c) {
   const int64_t nblk = ceil_div(c.T * c.k, kAssignBlock);

@@ -387,6 +387,42 @@ def test_layer_small_cases(moe, cuda_device, case):
         assert_close(v["ye"][e, :n], r["ye"][e, :n], what=f"ye[{e}]", **tol)
 
 
+@pytest.mark.parametrize("k", [1, 2])
+def test_fused_router_exact_ties(moe, cuda_device, k):
+    """Duplicated router rows give exactly tied logits; the router's fused top-k
+    must resolve them to the lower expert index, as the oracle does."""
+    dev = cuda_device
+    T, d, f, E = 777, 128, 128, 48
+    x = synth.normal(13, 1, (T, d), 1.0, torch.bfloat16)
+    Wr = synth.normal(13, 2, (E, d), 1.0 / math.sqrt(d), torch.float32)
+    Wr[5] = Wr[3] * 3.0   # experts 3 < 5 < 9 share one row that often wins
+    Wr[3] = Wr[5]
+    Wr[9] = Wr[5]
+    Wr[40] = Wr[12]
+    Wr = Wr.to(torch.bfloat16)
+    W1 = synth.normal(13, 3, (E, f, d), 0.02, torch.bfloat16)
+    W2 = synth.normal(13, 4, (E, d, f), 0.02, torch.bfloat16)
+    C = oracle.capacity(T, E, 2.0)
+    cfg = moe.make_config(T, d, f, E, k, C, dtype=torch.bfloat16)
+    ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    moe.layer_forward(cfg, x.to(dev), W1.to(dev), W2.to(dev), Wr=Wr.to(dev), workspace=ws)
+    torch.cuda.synchronize()
+    v = moe.workspace_views(cfg, ws)
+    logits = oracle.router(x, Wr)
+    idx, gate = oracle.gate_topk(logits, k)
+    top = torch.topk(logits.double(), k + 1, dim=1).values
+    gaps = top[:, :-1] - top[:, 1:]
+    near = ((gaps > 0) & (gaps < 1e-5)).any(1)  # inexact near-ties may round either way
+    got = v["expert_idx"].cpu()
+    exact_tie = (gaps == 0).any(1)
+    assert int(exact_tie.sum()) > 50, "the duplicated rows should produce many exact ties"
+    ok = (got == idx).all(1) | near
+    assert bool(ok.all()), torch.nonzero(~ok).flatten()[:10]
+    same = (got == idx).all(1)
+    g = v["gate"].cpu().double()[same]
+    assert bool(((g - gate.double()[same]).abs() <= 1e-5 * gate.double()[same]).all())
+
+
 def test_layer_zero_tokens(moe, cuda_device):
     dev = cuda_device
     cfg = moe.make_config(0, 64, 64, 16, 1, 0, dtype=torch.bfloat16)
