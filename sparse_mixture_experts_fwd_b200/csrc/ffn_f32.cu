@@ -15,6 +15,8 @@ template <bool RELU>
 __global__ void __launch_bounds__(kTile * kTile) grouped_gemm_f32_kernel(
     int N, int K, int C, const int32_t* __restrict__ rows_per_group, const float* __restrict__ A,
     const float* __restrict__ B, float* __restrict__ out) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   const int g = blockIdx.z;
   int rows = __ldg(rows_per_group + g);
   rows = rows < 0 ? 0 : (rows > C ? C : rows);
@@ -49,14 +51,14 @@ int32_t launch_ffn_f32(const moe_config& c, const void* xe, const void* W1, cons
   const dim3 block(kTile, kTile);
   const unsigned my = static_cast<unsigned>((c.capacity + kTile - 1) / kTile);
   dim3 g1((c.d_ff + kTile - 1) / kTile, my, c.E);
-  grouped_gemm_f32_kernel<true><<<g1, block, 0, s>>>(c.d_ff, c.d_model, c.capacity, kept_cnt,
+  launch_pdl(grouped_gemm_f32_kernel<true>, dim3(g1), dim3(block), 0, s, c.d_ff, c.d_model, c.capacity, kept_cnt,
                                                      static_cast<const float*>(xe),
                                                      static_cast<const float*>(W1),
                                                      static_cast<float*>(H));
   int32_t rc = check_launch("grouped_gemm_f32_kernel (W1)");
   if (rc != MOE_OK) return rc;
   dim3 g2((c.d_model + kTile - 1) / kTile, my, c.E);
-  grouped_gemm_f32_kernel<false><<<g2, block, 0, s>>>(c.d_model, c.d_ff, c.capacity, kept_cnt,
+  launch_pdl(grouped_gemm_f32_kernel<false>, dim3(g2), dim3(block), 0, s, c.d_model, c.d_ff, c.capacity, kept_cnt,
                                                       static_cast<const float*>(H),
                                                       static_cast<const float*>(W2),
                                                       static_cast<float*>(ye));

@@ -154,21 +154,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
   sc.prefix = s_prefix;
   sc.units = E + p.lag;
 
-  for (int e = tid; e < E; e += kThreads) {
-    int r = p.kept_cnt[e];
-    r = r < 0 ? 0 : (r > p.C ? p.C : r);
-    s_rows[e] = r;
-    s_mblk[e] = (r + kBM - 1) / kBM;
-  }
-  if (tid == 0) s_abort = 0;
-  __syncthreads();
+  dev::pdl_trigger();
   if (tid == 0) {
-    int acc = 0;
-    for (int u = 0; u < sc.units; ++u) {
-      s_prefix[u] = acc;
-      acc += sc.g1(u) + sc.g2(u);
-    }
-    s_prefix[sc.units] = acc;
+    s_abort = 0;
     for (int s = 0; s < kStages; ++s) {
       dev::mbar_init(&full_bar[s], 1);
       dev::mbar_init(&empty_bar[s], 1);
@@ -193,6 +181,22 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
   if (warp == 1) {
     dev::tmem_alloc(&s_tmem_base, kTmemCols);
     dev::tmem_relinquish();
+  }
+  dev::pdl_wait();  // kept counts, xe and the zeroed counters are visible from here
+  for (int e = tid; e < E; e += kThreads) {
+    int r = p.kept_cnt[e];
+    r = r < 0 ? 0 : (r > p.C ? p.C : r);
+    s_rows[e] = r;
+    s_mblk[e] = (r + kBM - 1) / kBM;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int u = 0; u < sc.units; ++u) {
+      s_prefix[u] = acc;
+      acc += sc.g1(u) + sc.g2(u);
+    }
+    s_prefix[sc.units] = acc;
   }
   dev::tc_fence_before();
   __syncthreads();
@@ -463,7 +467,7 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
     return check_launch("cudaFuncSetAttribute(ffn_tc_kernel)");
   const int64_t max_tiles = E * mblk_max * (nb1 + nb2);
   const int grid = static_cast<int>(std::min<int64_t>(sms, max_tiles));
-  ffn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tx, tw1, th, tw2, p);
+  launch_pdl(ffn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, tx, tw1, th, tw2, p);
   return check_launch("ffn_tc_kernel");
 }
 

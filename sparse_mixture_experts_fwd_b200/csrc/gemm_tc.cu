@@ -117,26 +117,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int n_blocks = (p.N + BN - 1) / BN;
   const int num_kb = p.K / kBK;
 
-  // ---- set-up: per-group tile counts, barriers, TMEM ----
-  for (int g = tid; g < G; g += kThreads) {
-    int r = p.group_rows ? p.group_rows[g] : p.fixed_rows;
-    r = r < 0 ? 0 : (r > p.max_rows ? p.max_rows : r);
-    s_rows[g] = r;
-    s_mblk[g] = (r + kBM - 1) / kBM;
-  }
-  if (tid == 0) s_abort = 0;
-  if (p.clear && blockIdx.x == 0)
-    for (int i = tid; i < p.n_clear; i += kThreads) p.clear[i] = 0u;
-  if constexpr (EPI == EPI_TOPK)
-    for (int i = tid; i < BN; i += kThreads) s_bias[i] = (p.bias && i < p.N) ? p.bias[i] : 0.f;
-  __syncthreads();
+  // ---- set-up: barriers and TMEM (no global memory), then per-group tile counts ----
+  dev::pdl_trigger();
   if (tid == 0) {
-    int acc = 0;
-    for (int g = 0; g < G; ++g) {
-      s_prefix[g] = acc;
-      acc += s_mblk[g] * n_blocks;
-    }
-    s_prefix[G] = acc;
+    s_abort = 0;
     for (int s = 0; s < S; ++s) {
       dev::mbar_init(&full_bar[s], 1);
       dev::mbar_init(&empty_bar[s], 1);
@@ -155,6 +139,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 1) {
     dev::tmem_alloc(&s_tmem_base, C::kTmemCols);
     dev::tmem_relinquish();
+  }
+  dev::pdl_wait();  // the previous kernel's outputs (row counts, x) are visible from here
+  for (int g = tid; g < G; g += kThreads) {
+    int r = p.group_rows ? p.group_rows[g] : p.fixed_rows;
+    r = r < 0 ? 0 : (r > p.max_rows ? p.max_rows : r);
+    s_rows[g] = r;
+    s_mblk[g] = (r + kBM - 1) / kBM;
+  }
+  if (p.clear && blockIdx.x == 0)
+    for (int i = tid; i < p.n_clear; i += kThreads) p.clear[i] = 0u;
+  if constexpr (EPI == EPI_TOPK)
+    for (int i = tid; i < BN; i += kThreads) s_bias[i] = (p.bias && i < p.N) ? p.bias[i] : 0.f;
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int g = 0; g < G; ++g) {
+      s_prefix[g] = acc;
+      acc += s_mblk[g] * n_blocks;
+    }
+    s_prefix[G] = acc;
   }
   dev::tc_fence_before();
   __syncthreads();
@@ -446,7 +450,7 @@ int32_t launch_gemm(const void* A, uint64_t a_rows, const void* B, uint64_t b_ro
       cudaSuccess)
     return check_launch("cudaFuncSetAttribute(gemm_tc_kernel)");
   int grid = static_cast<int>(max_tiles < num_sms() ? max_tiles : num_sms());
-  kern<<<grid, kThreads, C::kSmemBytes, s>>>(ta, tb, p);
+  launch_pdl(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, ta, tb, p);
   return check_launch("gemm_tc_kernel");
 }
 

@@ -23,6 +23,23 @@ int32_t check_launch(const char* what);  // maps cudaGetLastError to MOE_ERR_CUD
 int num_sms();                            // SM count of the current device (cached)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launch `kern` with programmatic stream serialisation (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 inline size_t elem_size(int32_t dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -89,6 +106,14 @@ MOE_DEV uint32_t smem_u32(const void* p) {
 }
 
 MOE_DEV uint32_t lane_id() { return threadIdx.x & 31u; }
+
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation: it lets the next kernel start
+// early (pdl_trigger at entry) and performs pdl_wait, which returns once the
+// previous kernel on the stream has completed and its writes are visible,
+// before its first global-memory read or write.
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // -- mbarrier --
 MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {

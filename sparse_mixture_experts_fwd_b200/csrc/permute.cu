@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
                                                        uint4* __restrict__ xe,
                                                        unsigned int* __restrict__ zero_words,
                                                        int n_zero) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   // counters the next kernel on this stream expects at zero (the fused expert FFN)
@@ -94,6 +96,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int row_vec, in
                                                       const int32_t* __restrict__ slot,
                                                       const uint8_t* __restrict__ kept,
                                                       uint4* __restrict__ y) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   constexpr int N = V::kN;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -150,11 +154,11 @@ int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* exper
   const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
   const unsigned grid = grid_for_tokens(c.T);
   if (c.k == 1)
-    dispatch_kernel<1><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
+    launch_pdl(dispatch_kernel<1>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
                                             expert_idx, slot, kept, static_cast<uint4*>(xe),
                                             zero_words, n_zero);
   else
-    dispatch_kernel<2><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
+    launch_pdl(dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
                                             expert_idx, slot, kept, static_cast<uint4*>(xe),
                                             zero_words, n_zero);
   return check_launch("dispatch_kernel");
@@ -170,17 +174,17 @@ int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* exper
   uint4* yv = static_cast<uint4*>(y);
   if (c.dtype == MOE_DTYPE_BF16) {
     if (c.k == 1)
-      combine_kernel<1, Bf16x8><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, yev, expert_idx,
+      launch_pdl(combine_kernel<1, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
                                                      gate, slot, kept, yv);
     else
-      combine_kernel<2, Bf16x8><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, yev, expert_idx,
+      launch_pdl(combine_kernel<2, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
                                                      gate, slot, kept, yv);
   } else {
     if (c.k == 1)
-      combine_kernel<1, F32x4><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, yev, expert_idx,
+      launch_pdl(combine_kernel<1, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
                                                     gate, slot, kept, yv);
     else
-      combine_kernel<2, F32x4><<<grid, 256, 0, s>>>(c.T, row_vec, c.capacity, yev, expert_idx,
+      launch_pdl(combine_kernel<2, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
                                                     gate, slot, kept, yv);
   }
   return check_launch("combine_kernel");

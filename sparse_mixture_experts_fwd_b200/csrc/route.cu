@@ -49,6 +49,8 @@ __device__ __forceinline__ void clear_flags(unsigned int* flags, int nblk) {
 __global__ void router_f32_kernel(int64_t T, int d, int E, const float* __restrict__ x,
                                   const float* __restrict__ Wr, const float* __restrict__ bias,
                                   float* __restrict__ logits) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (i >= T * E) return;
   const int64_t t = i / E;
@@ -80,6 +82,8 @@ __global__ void __launch_bounds__(256) gate_topk_kernel(int64_t T, int E,
                                                         int32_t* __restrict__ expert_idx,
                                                         float* __restrict__ gate,
                                                         unsigned int* flags, int nblk) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   clear_flags(flags, nblk);
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -134,6 +138,8 @@ __global__ void route_rre_kernel(int64_t T, int E, int G, uint64_t seed,
                                  const int32_t* __restrict__ domain,
                                  int32_t* __restrict__ expert_idx, float* __restrict__ gate,
                                  int32_t* status, unsigned int* flags, int nblk) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   clear_flags(flags, nblk);
   const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (t >= T) return;
@@ -182,7 +188,9 @@ __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArg
   const int E = p.E;
 
   // 1. ranks inside the block
+  dev::pdl_trigger();
   for (int i = tid; i < 32 * E; i += kAssignBlock) s_cnt[i] = 0;
+  dev::pdl_wait();
   __syncthreads();
   const int64_t a = static_cast<int64_t>(b) * kAssignBlock + tid;
   int e = a < p.n_assign ? __ldg(p.expert_idx + a) : -1;
@@ -293,6 +301,8 @@ __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArg
 // Totals for a call with no choices (T = 0): zero counts, empty row map.
 __global__ void assign_empty_kernel(int E, int C, int32_t* arrivals, int32_t* kept_cnt,
                                     int32_t* n_dropped, int32_t* tok_of_row) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
   for (int x = threadIdx.x; x < E; x += blockDim.x) {
     arrivals[x] = 0;
     kept_cnt[x] = 0;
@@ -321,9 +331,9 @@ int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, co
                           float* logits, cudaStream_t s) {
   const int64_t n = c.T * c.E;
   if (n == 0) return MOE_OK;
-  router_f32_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, s>>>(
-      c.T, c.d_model, c.E, static_cast<const float*>(x), static_cast<const float*>(Wr), bias,
-      logits);
+  launch_pdl(router_f32_kernel, dim3(static_cast<unsigned>(ceil_div(n, 256))), dim3(256), 0, s,
+             c.T, c.d_model, c.E, static_cast<const float*>(x), static_cast<const float*>(Wr),
+             bias, logits);
   return check_launch("router_f32_kernel");
 }
 
@@ -341,24 +351,24 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
   int32_t* aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
   int32_t* incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
   if (T == 0) {
-    assign_empty_kernel<<<1, 256, 0, s>>>(c.E, c.capacity, arrivals, kept_cnt, n_dropped,
+    launch_pdl(assign_empty_kernel, dim3(1), dim3(256), 0, s, c.E, c.capacity, arrivals, kept_cnt, n_dropped,
                                           tok_of_row);
     return check_launch("assign_empty_kernel");
   }
   if (c.mode == MOE_ROUTE_TOPK) {
     const int64_t blocks = std::min<int64_t>(ceil_div(T, 8), int64_t(num_sms()) * 16);
     if (c.k == 1)
-      gate_topk_kernel<1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-          T, c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
+      launch_pdl(gate_topk_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
+                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
     else
-      gate_topk_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-          T, c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
+      launch_pdl(gate_topk_kernel<2>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
+                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
     int32_t rc = check_launch("gate_topk_kernel");
     if (rc != MOE_OK) return rc;
   } else {
-    route_rre_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, s>>>(
-        T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status, flags,
-        static_cast<int>(nblk));
+    launch_pdl(route_rre_kernel, dim3(static_cast<unsigned>(ceil_div(T, 256))), dim3(256), 0, s,
+               T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status, flags,
+               static_cast<int>(nblk));
     int32_t rc = check_launch("route_rre_kernel");
     if (rc != MOE_OK) return rc;
   }
@@ -374,7 +384,7 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
   const int64_t n_assign = c.T * c.k;
   const int64_t nblk = ceil_div(n_assign, kAssignBlock);
   if (nblk == 0) {
-    assign_empty_kernel<<<1, 256, 0, s>>>(c.E, c.capacity, arrivals, kept_cnt, n_dropped,
+    launch_pdl(assign_empty_kernel, dim3(1), dim3(256), 0, s, c.E, c.capacity, arrivals, kept_cnt, n_dropped,
                                           tok_of_row);
     return check_launch("assign_empty_kernel");
   }
@@ -399,7 +409,7 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
   p.incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
   p.status = status;
   const size_t smem = (33 * static_cast<size_t>(c.E)) * sizeof(int);
-  assign_kernel<<<static_cast<unsigned>(nblk), kAssignBlock, smem, s>>>(p);
+  launch_pdl(assign_kernel, dim3(static_cast<unsigned>(nblk)), dim3(kAssignBlock), smem, s, p);
   return check_launch("assign_kernel");
 }
 
