@@ -426,6 +426,12 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
                       int32_t* status, cudaStream_t s) {
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
+  if (C >= 512) {
+    // Experts with hundreds of rows make the GEMMs tensor-core bound; SM
+    // pairs (256 x 256 tiles, cta_group::2) feed each SM a third fewer operand
+    // bytes per flop than single-CTA 128 x 256 tiles.
+    return launch_ffn_pairs(c, xe, W1, W2, kept_cnt, H, ye, status, s);
+  }
   if (C > kBM) {
     // Experts span several 128-row blocks: several CTAs share each weight
     // tile, and the two-launch kernels, whose static tile order keeps those

@@ -52,6 +52,9 @@ int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, co
 int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1, const void* W2,
                             const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
                             cudaStream_t s);
+int32_t launch_ffn_pairs(const moe_config& c, const void* xe, const void* W1, const void* W2,
+                         const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
+                         cudaStream_t s);
 // sync: ffn_sync_bytes(c) bytes of scratch; sync_zeroed says the caller
 // already zeroed it on this stream (else the launcher does).
 size_t ffn_sync_bytes(const moe_config& c);

@@ -196,6 +196,8 @@ def test_combine(moe, cuda_device, case):
 FFN_SHAPES = {
     # C > 128: the two-launch grouped GEMM
     "multi_block": (5, 300, 256, 768, [300, 0, 129, 1, 128]),
+    # C >= 512: SM pairs (cta_group::2, 256-row tiles; CTA 1's half empty for small experts)
+    "sm_pairs": (6, 512, 256, 512, [512, 0, 257, 256, 1, 300]),
     # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
     "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
 }
