@@ -322,9 +322,16 @@ def run_b200(args, w, world, rank, local):
     ffn_bytes = 2 * w.E * w.d_model * w.d_ff * es + 2 * n_kept * w.d_model * es
     ffn_flops = 4.0 * n_kept * w.d_model * w.d_ff
     ffn_s = stage_ms["expert_ffn"] / 1e3
+    # top-1 bf16 layers combine inside the expert FFN (its GEMM-2 epilogue writes
+    # gate * row to y); the dispatch kernel then also zeroes the dropped tokens' rows
+    fused_combine = w.k == 1 and w.dtype == "bf16"
     disp_bytes = (tok_any + n_kept) * w.d_model * es + 9 * w.T * w.k
-    comb_bytes = (n_kept + w.T) * w.d_model * es + 9 * w.T * w.k
-    dc_s = (stage_ms["dispatch"] + stage_ms["combine"]) / 1e3
+    if fused_combine:
+        disp_bytes += (w.T - tok_any) * w.d_model * es
+        comb_bytes = 0
+    else:
+        comb_bytes = (n_kept + w.T) * w.d_model * es + 9 * w.T * w.k
+    dc_s = (stage_ms["dispatch"] + (0.0 if fused_combine else stage_ms["combine"])) / 1e3
     intensity = ffn_flops / ffn_bytes
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if intensity < ridge:
@@ -427,6 +434,7 @@ def run_b200(args, w, world, rank, local):
         "stages_ms": {k: round(v_, 5) for k, v_ in stage_ms.items()},
         "expert_ffn_tflops": ffn_flops / ffn_s / 1e12,
         "dispatch_combine_gbs": (disp_bytes + comb_bytes) / dc_s / 1e9,
+        "combine": "fused into the expert FFN's GEMM-2 epilogue" if fused_combine else "kernel",
         "routing": {"n_kept": n_kept, "n_dropped": n_dropped,
                     "drop_rate": n_dropped / (w.T * w.k)},
         "gpu_launches": launches_per_step * args.steps,

@@ -194,7 +194,10 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert
  * dispatch -> expert FFN -> combine, all on `stream`.  Wr (+ bias) for TOPK,
  * domain_id for RRE (the other may be null).  y [T, d] in cfg->dtype.
  * workspace: moe_workspace_size(cfg) bytes laid out as moe_workspace_layout
- * describes; it holds every intermediate after the call.
+ * describes; it holds the intermediates after the call, except that bf16
+ * layers fuse the gate into the router (no logits) and bf16 top-1 layers
+ * fuse the combine into the expert FFN, which writes gate * E(x) straight
+ * to y (ye is left untouched).
  * stage_events (nullable; a profiling hook): host array of 6 cudaEvent_t
  * (entries may be null) recorded on `stream` before the router and after
  * the router, the assignment, the dispatch, the expert FFN and the combine. */

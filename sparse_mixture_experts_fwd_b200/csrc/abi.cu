@@ -353,14 +353,21 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
     MOE_TRY(launch_route_assign(c, logits, domain_id, expert_idx, gate, slot, kept, tok_of_row,
                                 arrivals, kept_cnt, n_dropped, scratch, status, s));
   MOE_TRY(mark(2));
+  // Top-1 bf16 layers combine inside the expert FFN: its second GEMM writes
+  // gate * row straight into y (token order) and the dispatch kernel zeroes the
+  // rows of dropped tokens, so ye is not materialised and no combine runs.
+  const bool fused_combine = c.k == 1 && c.dtype == MOE_DTYPE_BF16 && c.T > 0;
+  const Top1Out top1{tok_of_row, gate, y};
   MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, s,
-                          dispatch_zeroes ? ffn_sync : nullptr, dispatch_zeroes ? n_sync_words : 0));
+                          dispatch_zeroes ? ffn_sync : nullptr, dispatch_zeroes ? n_sync_words : 0,
+                          fused_combine ? y : nullptr));
   MOE_TRY(mark(3));
   if (c.dtype == MOE_DTYPE_BF16)
-    MOE_TRY(launch_ffn_tc(c, xe, W1, W2, kept_cnt, H, ye, ffn_sync, dispatch_zeroes, status, s));
+    MOE_TRY(launch_ffn_tc(c, xe, W1, W2, kept_cnt, H, ye, ffn_sync, dispatch_zeroes, status, s,
+                          fused_combine ? &top1 : nullptr));
   else MOE_TRY(launch_ffn_f32(c, xe, W1, W2, kept_cnt, H, ye, s));
   MOE_TRY(mark(4));
-  MOE_TRY(launch_combine(c, ye, expert_idx, gate, slot, kept, y, s));
+  if (!fused_combine) MOE_TRY(launch_combine(c, ye, expert_idx, gate, slot, kept, y, s));
   return mark(5);
 }
 

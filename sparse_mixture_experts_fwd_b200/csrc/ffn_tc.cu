@@ -54,6 +54,11 @@ struct FfnParams {
   unsigned int* tile_ctr;  // zero before launch
   unsigned int* done1;     // [E], zero before launch
   int32_t* status;
+  // top-1 layers: GEMM 2 writes gate * row straight to y [T, d] in token order
+  // (ye untouched); null -> write ye
+  const int32_t* tok_of_row;
+  const float* gate;
+  __nv_bfloat16* y;
 };
 
 struct Tile {
@@ -330,6 +335,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       const int64_t grow = static_cast<int64_t>(x.e) * p.C + x.m * kBM + row_local;
       const int N = x.kind == 1 ? p.f : p.d;
       __nv_bfloat16* out = (x.kind == 1 ? p.H : p.ye) + grow * N;
+      float scale = 1.f;
+      if (x.kind == 2 && p.y && row_ok) {
+        // top-1 combine (eq. 2 with one expert): y[t] = gate_t * E(x_t), into token order
+        const int tok = __ldg(p.tok_of_row + grow);
+        scale = __ldg(p.gate + tok);
+        out = p.y + static_cast<int64_t>(tok) * N;
+      }
       const int n0 = x.n * kBN;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * kAccStride);
@@ -344,8 +356,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float a = __uint_as_float(r[2 * i]);
-            float b = __uint_as_float(r[2 * i + 1]);
+            float a = __uint_as_float(r[2 * i]) * scale;
+            float b = __uint_as_float(r[2 * i + 1]) * scale;
             if (relu) { a = fmaxf(a, 0.f); b = fmaxf(b, 0.f); }
             __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             packed[i] = *reinterpret_cast<uint32_t*>(&h);
@@ -423,21 +435,21 @@ size_t ffn_sync_bytes(const moe_config& c) {
 
 int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const void* W2,
                       const int32_t* kept_cnt, void* H, void* ye, void* sync, bool sync_zeroed,
-                      int32_t* status, cudaStream_t s) {
+                      int32_t* status, cudaStream_t s, const Top1Out* top1) {
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
   if (C >= 512) {
     // Experts with hundreds of rows make the GEMMs tensor-core bound; SM
     // pairs (256 x 256 tiles, cta_group::2) feed each SM a third fewer operand
     // bytes per flop than single-CTA 128 x 256 tiles.
-    return launch_ffn_pairs(c, xe, W1, W2, kept_cnt, H, ye, status, s);
+    return launch_ffn_pairs(c, xe, W1, W2, kept_cnt, H, ye, status, s, top1);
   }
   if (C > kBM) {
     // Experts span several 128-row blocks: several CTAs share each weight
     // tile, and the two-launch kernels, whose static tile order keeps those
     // CTAs in lockstep, measured faster (fewer L2 reads, higher clocks under
     // the power cap).  The fused kernel wins when each weight tile has one user.
-    return launch_ffn_two_pass(c, xe, W1, W2, kept_cnt, H, ye, status, s);
+    return launch_ffn_two_pass(c, xe, W1, W2, kept_cnt, H, ye, status, s, top1);
   }
   if (!sync_zeroed) {
     cudaError_t e = cudaMemsetAsync(sync, 0, ffn_sync_bytes(c), s);
@@ -468,6 +480,11 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
   p.tile_ctr = static_cast<unsigned int*>(sync);
   p.done1 = static_cast<unsigned int*>(sync) + 1;
   p.status = status;
+  if (top1) {
+    p.tok_of_row = top1->tok_of_row;
+    p.gate = top1->gate;
+    p.y = static_cast<__nv_bfloat16*>(top1->y);
+  }
   if (cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes) != cudaSuccess)
     return check_launch("cudaFuncSetAttribute(ffn_tc_kernel)");

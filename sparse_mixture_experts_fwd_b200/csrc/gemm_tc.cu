@@ -53,6 +53,9 @@ struct GemmParams {
   float* gate;                 // EPI_TOPK: [T, k]
   unsigned int* clear;         // nullable: words block 0 zeroes for the next kernel
   int n_clear;
+  const int32_t* scatter_tok;  // EPI_BF16, top-1 layers: row -> token map, or null
+  const float* scatter_gate;   //   gate per token
+  __nv_bfloat16* scatter_y;    //   y [T, out_ld] written instead of out
   int32_t* status;             // nullable
 };
 
@@ -359,6 +362,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       } else {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.out_ld;
+        float scale = 1.f;
+        if (EPI == EPI_BF16 && p.scatter_y && row_ok) {
+          // top-1 combine: y[t] = gate_t * row, written in token order
+          const int tok = __ldg(p.scatter_tok + grow);
+          scale = __ldg(p.scatter_gate + tok);
+          out = p.scatter_y + static_cast<int64_t>(tok) * p.out_ld;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -369,8 +379,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t packed[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float a = __uint_as_float(r[2 * i]);
-              float b = __uint_as_float(r[2 * i + 1]);
+              float a = __uint_as_float(r[2 * i]) * scale;
+              float b = __uint_as_float(r[2 * i + 1]) * scale;
               if (EPI == EPI_RELU_BF16) { a = fmaxf(a, 0.f); b = fmaxf(b, 0.f); }
               __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
               packed[i] = *reinterpret_cast<uint32_t*>(&h);
@@ -461,7 +471,7 @@ int32_t launch_gemm(const void* A, uint64_t a_rows, const void* B, uint64_t b_ro
 // share a weight tile in lockstep, so its k-slices are served once from L2.
 int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1, const void* W2,
                             const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                            cudaStream_t s) {
+                            cudaStream_t s, const Top1Out* top1) {
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
   const int64_t mblk_max = (C + kBM - 1) / kBM;
@@ -488,6 +498,11 @@ int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1,
   p.K = c.d_ff;
   p.out = ye;
   p.out_ld = d;
+  if (top1) {
+    p.scatter_tok = top1->tok_of_row;
+    p.scatter_gate = top1->gate;
+    p.scatter_y = static_cast<__nv_bfloat16*>(top1->y);
+  }
   return launch_gemm<256, EPI_BF16>(H, E * C, W2, E * d, p, E * mblk_max * ((d + 255) / 256), s);
 }
 

@@ -55,6 +55,9 @@ struct Gemm2Params {
   __nv_bfloat16* out;
   int64_t out_ld;
   int32_t* status;
+  const int32_t* scatter_tok;  // EPI2_BF16, top-1 layers: row -> token map, or null
+  const float* scatter_gate;   //   gate per token
+  __nv_bfloat16* scatter_y;    //   y [T, out_ld] written instead of out
 };
 
 MOE_DEV uint32_t cta_rank() {
@@ -291,6 +294,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool row_ok = row_in_group < s_rows[tc.g];
       const int64_t grow = static_cast<int64_t>(tc.g) * p.a_group_rows + row_in_group;
       __nv_bfloat16* out = p.out + grow * p.out_ld;
+      float scale = 1.f;
+      if (EPI == EPI2_BF16 && p.scatter_y && row_ok) {
+        // top-1 combine: y[t] = gate_t * row, written in token order
+        const int tok = __ldg(p.scatter_tok + grow);
+        scale = __ldg(p.scatter_gate + tok);
+        out = p.scatter_y + static_cast<int64_t>(tok) * p.out_ld;
+      }
       const int n0 = tc.n * kBN;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * kAccStride);
@@ -304,8 +314,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float a = __uint_as_float(r[2 * i]);
-            float b = __uint_as_float(r[2 * i + 1]);
+            float a = __uint_as_float(r[2 * i]) * scale;
+            float b = __uint_as_float(r[2 * i + 1]) * scale;
             if (EPI == EPI2_RELU_BF16) { a = fmaxf(a, 0.f); b = fmaxf(b, 0.f); }
             __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             packed[i] = *reinterpret_cast<uint32_t*>(&h);
@@ -409,7 +419,7 @@ int32_t launch_pair(const void* A, uint64_t a_rows, const void* B, uint64_t b_ro
 // H = ReLU(xe W1^T), ye = H W2^T on SM pairs, 256 x 256 tiles.
 int32_t launch_ffn_pairs(const moe_config& c, const void* xe, const void* W1, const void* W2,
                          const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                         cudaStream_t s) {
+                         cudaStream_t s, const Top1Out* top1) {
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
   const int64_t mblk_max = (C + kBM - 1) / kBM;
@@ -432,6 +442,11 @@ int32_t launch_ffn_pairs(const moe_config& c, const void* xe, const void* W1, co
   p.K = c.d_ff;
   p.out = static_cast<__nv_bfloat16*>(ye);
   p.out_ld = d;
+  if (top1) {
+    p.scatter_tok = top1->tok_of_row;
+    p.scatter_gate = top1->gate;
+    p.scatter_y = static_cast<__nv_bfloat16*>(top1->y);
+  }
   return launch_pair<EPI2_BF16>(H, E * C, W2, E * d, p, E * mblk_max * ((d + kBN - 1) / kBN), s);
 }
 

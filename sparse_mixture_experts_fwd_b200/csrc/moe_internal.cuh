@@ -49,18 +49,25 @@ int32_t launch_router_tc(const moe_config& c, const void* x, const void* Wr, con
                          float* logits, int32_t* status, cudaStream_t s);
 int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, const float* bias,
                           float* logits, cudaStream_t s);
+// Top-1 layers: the expert FFN's second GEMM writes y[t] = gate[t] * E(x_t)
+// directly in token order (row -> token map tok_of_row) instead of ye.
+struct Top1Out {
+  const int32_t* tok_of_row;
+  const float* gate;
+  void* y;
+};
 int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1, const void* W2,
                             const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                            cudaStream_t s);
+                            cudaStream_t s, const Top1Out* top1 = nullptr);
 int32_t launch_ffn_pairs(const moe_config& c, const void* xe, const void* W1, const void* W2,
                          const int32_t* kept_cnt, void* H, void* ye, int32_t* status,
-                         cudaStream_t s);
+                         cudaStream_t s, const Top1Out* top1 = nullptr);
 // sync: ffn_sync_bytes(c) bytes of scratch; sync_zeroed says the caller
 // already zeroed it on this stream (else the launcher does).
 size_t ffn_sync_bytes(const moe_config& c);
 int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const void* W2,
                       const int32_t* kept_cnt, void* H, void* ye, void* sync, bool sync_zeroed,
-                      int32_t* status, cudaStream_t s);
+                      int32_t* status, cudaStream_t s, const Top1Out* top1 = nullptr);
 int32_t launch_ffn_f32(const moe_config& c, const void* xe, const void* W1, const void* W2,
                        const int32_t* kept_cnt, void* H, void* ye, cudaStream_t s);
 int32_t launch_route_assign(const moe_config& c, const float* logits, const int32_t* domain,
@@ -78,10 +85,12 @@ int32_t launch_router_topk_tc(const moe_config& c, const void* x, const void* Wr
 int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* slot,
                       uint8_t* kept, int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
                       int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s);
-// zero_words (nullable): n_zero words the dispatch kernel clears for the next kernel
+// zero_words (nullable): n_zero words the dispatch kernel clears for the next kernel;
+// y_zero (nullable): y [T, d], whose rows of tokens with no kept choice it zeroes
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
                         const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
-                        unsigned int* zero_words = nullptr, int n_zero = 0);
+                        unsigned int* zero_words = nullptr, int n_zero = 0,
+                        void* y_zero = nullptr);
 int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* expert_idx,
                        const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
                        cudaStream_t s);

@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
                                                        const uint8_t* __restrict__ kept,
                                                        uint4* __restrict__ xe,
                                                        unsigned int* __restrict__ zero_words,
-                                                       int n_zero) {
+                                                       int n_zero, uint4* __restrict__ y_zero) {
   dev::pdl_trigger();
   dev::pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -43,7 +43,13 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
                      __ldg(slot + t * K + j)) * row_vec;
       }
     }
-    if (nd == 0) continue;
+    if (nd == 0) {
+      // top-1 layers combine inside the expert FFN, which writes only kept
+      // tokens; a dropped token's output row is 0 (drop rule)
+      if (y_zero)
+        for (int v = lane; v < row_vec; v += 32) y_zero[t * row_vec + v] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
     const uint4* src = x + t * row_vec;
 #pragma unroll 4
     for (int v = lane; v < row_vec; v += 32) {
@@ -149,18 +155,19 @@ unsigned grid_for_tokens(int64_t T) {
 
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
                         const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
-                        unsigned int* zero_words, int n_zero) {
-  if (c.T == 0 || c.capacity == 0) return MOE_OK;
+                        unsigned int* zero_words, int n_zero, void* y_zero) {
+  if (c.T == 0 || (c.capacity == 0 && !y_zero)) return MOE_OK;
   const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
   const unsigned grid = grid_for_tokens(c.T);
+  uint4* yz = static_cast<uint4*>(y_zero);
   if (c.k == 1)
-    launch_pdl(dispatch_kernel<1>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
-                                            expert_idx, slot, kept, static_cast<uint4*>(xe),
-                                            zero_words, n_zero);
+    launch_pdl(dispatch_kernel<1>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity,
+               static_cast<const uint4*>(x), expert_idx, slot, kept, static_cast<uint4*>(xe),
+               zero_words, n_zero, yz);
   else
-    launch_pdl(dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, static_cast<const uint4*>(x),
-                                            expert_idx, slot, kept, static_cast<uint4*>(xe),
-                                            zero_words, n_zero);
+    launch_pdl(dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity,
+               static_cast<const uint4*>(x), expert_idx, slot, kept, static_cast<uint4*>(xe),
+               zero_words, n_zero, yz);
   return check_launch("dispatch_kernel");
 }
 

@@ -310,8 +310,11 @@ def test_layer_forward_full(moe, cuda_device, case):
 
     with cf.ThreadPoolExecutor(max_workers=threads()) as ex:
         ye_ref = list(ex.map(one_row, rows))
+    # top-1 bf16 layers combine inside the expert FFN and never materialise ye
+    ye_kept = not (w.k == 1 and w.dtype == "bf16")
     for (t, e, s), yr in zip(rows, ye_ref):
-        assert_close(v["ye"][e, s], yr, what=f"ye[{e},{s}]")
+        if ye_kept:
+            assert_close(v["ye"][e, s], yr, what=f"ye[{e},{s}]")
         assert torch.equal(v["xe"][e, s].view(torch.int16) if w.dtype == "bf16" else v["xe"][e, s],
                            inp["x"][t].view(torch.int16) if w.dtype == "bf16" else inp["x"][t])
 
@@ -386,7 +389,8 @@ def test_layer_small_cases(moe, cuda_device, case):
     for e in range(E):
         n = int(r["kept_cnt"][e])
         assert_close(v["H"][e, :n], r["H"][e, :n], what=f"H[{e}]", **tol)
-        assert_close(v["ye"][e, :n], r["ye"][e, :n], what=f"ye[{e}]", **tol)
+        if not (k == 1 and dtype == "bf16"):  # top-1 bf16: combined in the FFN, no ye
+            assert_close(v["ye"][e, :n], r["ye"][e, :n], what=f"ye[{e}]", **tol)
 
 
 @pytest.mark.parametrize("k", [1, 2])
