@@ -33,6 +33,13 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+# DRAM bytes (read + write) of the expert-FFN stage per layer step, from one ncu
+# capture of the kernels as shipped (the profile named beside each number).
+# A workload without a capture of its current kernels reports null.
+FFN_TRAFFIC = {
+    "switch_base": (1242.1e6 + 29.3e6, "profiles/ffn_tc_switch_base.md"),
+    "xmoe_top2": (604.1e6 + 227.9e6 + 825.7e6 + 59.5e6, "profiles/gemm_pair_xmoe_top2.md"),
+}
 METRIC = "MoE-layer tokens/sec (1 B200); expert-FFN TFLOP/s; dispatch+combine GB/s"
 
 
@@ -341,7 +348,11 @@ def run_b200(args, w, world, rank, local):
         roof = {"bound": "tensor", "achieved": ffn_flops / ffn_s / 1e12,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    tr = FFN_TRAFFIC.get(w.name)
+    roof["traffic"] = tr[0] if tr else None
+    roof["traffic_unit"] = "bytes per expert-FFN stage (ncu dram__bytes_read + write)"
+    roof["traffic_source"] = tr[1] if tr else None
+    roof["algorithmic_bytes"] = ffn_bytes
     roof["kernel"] = ("expert FFN: " + (
         "grouped_gemm_f32_kernel x2" if w.dtype == "f32" else
         "ffn_tc_kernel x1 (both GEMMs fused)" if C <= 128 else
