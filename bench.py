@@ -224,6 +224,67 @@ def run_reference(args, w, world, rank):
 # the B200 arm
 # ---------------------------------------------------------------------------
 
+def kernel_launches(w, C):
+    """Kernels ``moe_layer_forward`` launches per step (T > 0), stage by stage."""
+    bf16 = w.dtype == "bf16"
+    if w.mode == "rre":
+        route = 2                       # RRE choice, slot assignment
+    elif bf16:
+        route = 2                       # router GEMM with gate/top-k epilogue, slot assignment
+    else:
+        route = 3                       # fp32 router, gate/top-k, slot assignment
+    ffn = 1 if (bf16 and C <= 128) else 2
+    combine = 0 if (bf16 and w.k == 1) else 1   # top-1 bf16: inside the FFN's GEMM 2
+    return route + 1 + ffn + combine
+
+
+def stage_work(w, C, es, n_kept, tok_any):
+    """Algorithmic bytes and flops of each stage of one layer step.
+
+    Bytes count each tensor the stage must read or write once (activations,
+    weights, routing arrays); H, the FFN's hidden activations, is
+    implementation traffic and is not counted.
+    """
+    T, d, f, E, k = w.T, w.d_model, w.d_ff, w.E, w.k
+    fused_combine = w.k == 1 and w.dtype == "bf16"
+    st = {}
+    assign_out = 5 * T * k + 4 * E * C + 8 * E   # slot, kept, row -> token map, counts
+    if w.mode == "rre":
+        st["router"] = (0, 0.0)
+        # domain ids in, expert index and gate out, then the assignment
+        st["route_assign"] = (4 * T + 8 * T * k + assign_out, 0.0)
+    elif w.dtype == "bf16":
+        # logits stay in TMEM: x, W_r (and bias) in, expert index and gate out
+        st["router"] = (T * d * es + E * d * es + (4 * E if w.hot_experts else 0) + 8 * T * k,
+                        2.0 * T * d * E)
+        st["route_assign"] = (4 * T * k + assign_out, 0.0)
+    else:
+        st["router"] = (T * d * es + E * d * es + 4 * T * E, 2.0 * T * d * E)
+        st["route_assign"] = (4 * T * E + 8 * T * k + assign_out, 0.0)
+    disp = (tok_any + n_kept) * d * es + 9 * T * k
+    if fused_combine:
+        disp += (T - tok_any) * d * es                    # dropped tokens' output rows zeroed
+    st["dispatch"] = (disp, 0.0)
+    st["expert_ffn"] = (2 * E * d * f * es + 2 * n_kept * d * es, 4.0 * n_kept * d * f)
+    st["combine"] = (0 if fused_combine else (n_kept + T) * d * es + 9 * T * k, 0.0)
+    return st
+
+
+def stage_roofline(st, stage_ms, peaks):
+    """Per stage: time at the roofline (the slower of bytes at HBM and flops at
+    the sustained bf16 peak) over the measured stage time."""
+    out = {}
+    for n, (b, fl) in st.items():
+        ms = stage_ms[n]
+        t_roof = max(b / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops_sustained"] * 1e12))
+        out[n] = {"ms": round(ms, 5), "bytes": b, "flops": fl,
+                  "bound": "tensor" if fl / (peaks["bf16_tflops_sustained"] * 1e12) >
+                  b / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                  "gbs": round(b / (ms / 1e3) / 1e9, 1) if ms > 0 else None,
+                  "frac": round(t_roof / (ms / 1e3), 3) if ms > 0 and (b or fl) else None}
+    return out
+
+
 def run_b200(args, w, world, rank, local):
     import sparse_mixture_experts_fwd_b200 as moe
 
@@ -262,10 +323,7 @@ def run_b200(args, w, world, rank, local):
                           domain_id=doms[i % n_rot], y=y, workspace=ws, status=status,
                           stream=stream, stage_events=evs)
 
-    # our kernels per step: router (top-k layers), gate or RRE + 3 assignment
-    # kernels, dispatch, expert FFN (1 fused launch when C <= 128, else 2), combine
-    ffn_launches = 2 if (w.dtype == "f32" or C > 128) else 1
-    launches_per_step = (1 if w.mode == "topk" else 0) + 4 + 1 + ffn_launches + 1
+    launches_per_step = kernel_launches(w, C)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -325,23 +383,18 @@ def run_b200(args, w, world, rank, local):
     n_dropped = int(asg["n_dropped"].item())
     tok_any = int((asg["kept"].cpu().sum(1) > 0).sum())
 
-    # algorithmic work of the dominant stage (expert FFN) and of dispatch + combine
-    ffn_bytes = 2 * w.E * w.d_model * w.d_ff * es + 2 * n_kept * w.d_model * es
-    ffn_flops = 4.0 * n_kept * w.d_model * w.d_ff
+    # algorithmic work of every stage; the expert FFN is the dominant one
+    st = stage_work(w, C, es, n_kept, tok_any)
+    stages = stage_roofline(st, stage_ms, peaks)
+    ffn_bytes, ffn_flops = st["expert_ffn"]
     ffn_s = stage_ms["expert_ffn"] / 1e3
     # top-1 bf16 layers combine inside the expert FFN (its GEMM-2 epilogue writes
     # gate * row to y); the dispatch kernel then also zeroes the dropped tokens' rows
     fused_combine = w.k == 1 and w.dtype == "bf16"
-    disp_bytes = (tok_any + n_kept) * w.d_model * es + 9 * w.T * w.k
-    if fused_combine:
-        disp_bytes += (w.T - tok_any) * w.d_model * es
-        comb_bytes = 0
-    else:
-        comb_bytes = (n_kept + w.T) * w.d_model * es + 9 * w.T * w.k
+    disp_bytes, comb_bytes = st["dispatch"][0], st["combine"][0]
     dc_s = (stage_ms["dispatch"] + (0.0 if fused_combine else stage_ms["combine"])) / 1e3
-    intensity = ffn_flops / ffn_bytes
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if intensity < ridge:
+    # the FFN runs inside a long step: the sustained bf16 figure is its tensor peak
+    if stages["expert_ffn"]["bound"] == "hbm":
         roof = {"bound": "hbm", "achieved": ffn_bytes / ffn_s / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     else:
@@ -356,7 +409,8 @@ def run_b200(args, w, world, rank, local):
     roof["kernel"] = ("expert FFN: " + (
         "grouped_gemm_f32_kernel x2" if w.dtype == "f32" else
         "ffn_tc_kernel x1 (both GEMMs fused)" if C <= 128 else
-        "gemm_tc_kernel x2 (H = ReLU(xe W1^T), ye = H W2^T)"))
+        "gemm_tc_kernel x2 (H = ReLU(xe W1^T), ye = H W2^T)" if C < 512 else
+        "gemm_pair_kernel x2 on SM pairs (H = ReLU(xe W1^T), ye = H W2^T)"))
     roof["peak_source"] = peaks["source"]
     roof["algorithmic_per_launch"] = (f"{ffn_bytes / 1e9:.4f} GB" if roof["bound"] == "hbm"
                                       else f"{ffn_flops / 1e12:.4f} TFLOP")
@@ -443,6 +497,9 @@ def run_b200(args, w, world, rank, local):
                          "both larger than the 126 MB L2"},
         "roofline": roof,
         "stages_ms": {k: round(v_, 5) for k, v_ in stage_ms.items()},
+        "stages": stages,
+        "stages_note": "stage times from events the library records between its stages "
+                       "(each record serialises the stream); frac = roofline time / stage time",
         "expert_ffn_tflops": ffn_flops / ffn_s / 1e12,
         "dispatch_combine_gbs": (disp_bytes + comb_bytes) / dc_s / 1e9,
         "combine": "fused into the expert FFN's GEMM-2 epilogue" if fused_combine else "kernel",
