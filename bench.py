@@ -415,6 +415,78 @@ def run_b200(args, w, world, rank, local):
     roof["algorithmic_per_launch"] = (f"{ffn_bytes / 1e9:.4f} GB" if roof["bound"] == "hbm"
                                       else f"{ffn_flops / 1e12:.4f} TFLOP")
 
+    # ---- Switch load-balancing loss + routing entropy (top-k layers) ----
+    # From the fp32 logits of this batch (moe_router); K back-to-back calls of
+    # the C entry point timed with events on the stream.  Each call reads the
+    # T x E logits once (two launches).
+    aux = None
+    if w.mode == "topk":
+        import ctypes
+        logits = moe.router(cfg, xs[0], Wr, bias, stream=stream)
+        aux_ws = torch.empty(max(256, moe.aux_workspace_size(cfg)), dtype=torch.uint8, device=dev)
+        aux_out = torch.empty(2, dtype=torch.float64, device=dev)
+        aux_args = (ctypes.byref(cfg), ctypes.c_void_p(logits.data_ptr()), 1e-2,
+                    ctypes.c_void_p(aux_out.data_ptr()), None, None,
+                    ctypes.c_void_p(aux_ws.data_ptr()), aux_ws.numel(),
+                    ctypes.c_void_p(stream.cuda_stream))
+        for _ in range(3):
+            assert moe.lib.moe_aux_loss(*aux_args) == 0
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            moe.lib.moe_aux_loss(*aux_args)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        aux_ms = a0.elapsed_time(a1) / args.steps
+        aux_bytes = w.T * w.E * 4
+        aux = {"ms": aux_ms, "bytes": aux_bytes, "gbs": aux_bytes / (aux_ms / 1e3) / 1e9,
+               "frac_hbm": aux_bytes / (peaks["hbm_gbs"] * 1e9) / (aux_ms / 1e3),
+               "loss": float(aux_out[0]), "entropy": float(aux_out[1]), "alpha": 1e-2,
+               "note": "moe_aux_loss on this batch's fp32 router logits, back-to-back calls"}
+
+    # ---- SparseClip norm and clipping step (workloads that carry gradients) ----
+    # The norm reads every gradient once; the clip reads them for the norm and
+    # then reads and writes them (coef ~ 1/2 on every call, so the write path
+    # runs each time).  Gradients total 2.35 GB for the X-MoE workload.
+    sclip = None
+    if w.clip_dense and rank == 0:
+        gd, gs = synth.sparseclip_inputs(w)
+        gd = [t.to(dev) for t in gd]
+        gs = [t.to(dev) for t in gs]
+        n_el = sum(t.numel() for t in gd + gs)
+        sc_ws = torch.empty(max(16, moe.sparseclip_workspace_size(len(gd), len(gs))),
+                            dtype=torch.uint8, device=dev)
+        sc_out = torch.empty(4, dtype=torch.float64, device=dev)
+        for _ in range(3):
+            moe.sparseclip_norm(gd, gs, w.E, out=sc_out, workspace=sc_ws, stream=stream)
+        torch.cuda.synchronize()
+        norm0 = float(sc_out[0])
+        reps = min(args.steps, 20)
+        c0, c1, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        c0.record(stream)
+        for _ in range(reps):
+            moe.sparseclip_norm(gd, gs, w.E, out=sc_out, workspace=sc_ws, stream=stream)
+        c1.record(stream)
+        for i in range(reps):
+            moe.sparseclip_clip(gd, gs, w.E, norm0 * 0.5 ** (i + 1), out=sc_out, workspace=sc_ws,
+                                stream=stream)
+        c2.record(stream)
+        torch.cuda.synchronize()
+        norm_ms = c0.elapsed_time(c1) / reps
+        clip_ms = c1.elapsed_time(c2) / reps
+        nb, cb = 4 * n_el, 12 * n_el
+        sclip = {"elements": n_el, "norm_ms": norm_ms, "norm_bytes": nb,
+                 "norm_gbs": nb / (norm_ms / 1e3) / 1e9,
+                 "norm_frac_hbm": nb / (peaks["hbm_gbs"] * 1e9) / (norm_ms / 1e3),
+                 "clip_ms": clip_ms, "clip_bytes": cb, "clip_gbs": cb / (clip_ms / 1e3) / 1e9,
+                 "clip_frac_hbm": cb / (peaks["hbm_gbs"] * 1e9) / (clip_ms / 1e3),
+                 "coef_last": float(sc_out[3]),
+                 "note": "sparseclip_norm, and sparseclip_clip (norm + in-place scale by ~1/2), "
+                         "back-to-back calls on the workload's fp32 gradients"}
+        del gd, gs
+        torch.cuda.empty_cache()
+
     # ---- e2e through moe_layer_forward with host buffers ----
     # Every step copies its batch from pinned host memory and its output back.
     # The copies run on two copy streams, double-buffered, so step i's
@@ -503,6 +575,8 @@ def run_b200(args, w, world, rank, local):
         "expert_ffn_tflops": ffn_flops / ffn_s / 1e12,
         "dispatch_combine_gbs": (disp_bytes + comb_bytes) / dc_s / 1e9,
         "combine": "fused into the expert FFN's GEMM-2 epilogue" if fused_combine else "kernel",
+        "aux_loss": aux,
+        "sparseclip": sclip,
         "routing": {"n_kept": n_kept, "n_dropped": n_dropped,
                     "drop_rate": n_dropped / (w.T * w.k)},
         "gpu_launches": launches_per_step * args.steps,

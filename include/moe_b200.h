@@ -128,6 +128,9 @@ size_t moe_ffn_workspace_size(const moe_config* cfg);
 int32_t moe_workspace_layout(const moe_config* cfg, moe_workspace_map* out);
 size_t moe_workspace_size(const moe_config* cfg); /* 0 if cfg is invalid */
 
+/* Bytes of scratch moe_aux_loss needs (0 if cfg is invalid). */
+size_t moe_aux_workspace_size(const moe_config* cfg);
+
 /* Bytes of scratch sparseclip_norm needs for this many tensors. */
 size_t sparseclip_workspace_size(int32_t n_dense, int32_t n_sparse);
 
@@ -206,6 +209,23 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
                           void* workspace, size_t workspace_bytes, int32_t* status,
                           void* const* stage_events, moe_stream_t stream);
 
+/* Switch auxiliary load-balancing loss and mean routing entropy (Switch
+ * notes sec. 2.2, "A Differentiable Load Balancing Loss", eqs. (4)-(6); the
+ * routing entropy the TorchScale review tracks), from router logits [T, E]
+ * fp32 (moe_router's output; cfg->mode must be MOE_ROUTE_TOPK):
+ *   p(x)   = softmax over all E experts of the token's logits (eq. 1)
+ *   f[i]   = (1/T) #{tokens : argmax p = i}, ties to the lower index (eq. 5)
+ *   P[i]   = (1/T) sum over tokens of p_i (eq. 6)
+ *   out[0] = alpha * E * sum_i f[i] P[i]                                (eq. 4)
+ *   out[1] = (1/T) sum over tokens of -sum_i p_i ln p_i
+ * The pages use alpha = 1e-2.  out [2], f [E], P [E]: device double (f and P
+ * nullable).  T = 0 gives zeros.  Softmax and entropy per token in fp32,
+ * sums over tokens in double, added in a fixed order (deterministic).
+ * workspace: moe_aux_workspace_size(cfg) bytes. */
+int32_t moe_aux_loss(const moe_config* cfg, const float* logits, double alpha, double* out,
+                     double* f, double* P, void* workspace, size_t workspace_bytes,
+                     moe_stream_t stream);
+
 /* SparseClip global gradient norm ("[Paper review] TorchScale", proposed
  * method): ||g||_2 = ||(g_d, kappa g_s)||_2 with kappa = 1/sqrt(num_experts),
  *   out[0] = sqrt(Sd + Ss / num_experts), out[1] = Sd, out[2] = Ss,
@@ -219,6 +239,21 @@ int32_t sparseclip_norm(const float* const* dense, const int64_t* dense_len, int
                         const float* const* sparse, const int64_t* sparse_len, int32_t n_sparse,
                         int32_t num_experts, double* out, void* workspace, size_t workspace_bytes,
                         moe_stream_t stream);
+
+/* SparseClip clipping step (TorchScale review, proposed method: gradient
+ * clipping by the reweighted L2 norm ||(g_d, kappa g_s)||_2, kappa = 1/sqrt(E)):
+ * computes the norm exactly as sparseclip_norm (out[0..2]), then scales
+ * every dense and expert tensor IN PLACE by
+ *   coef = min(1, max_norm / norm)      (1 when norm <= max_norm: nothing written)
+ * and writes coef to out[3].  kappa only reweights the norm; the same coef
+ * applies to all tensors.  max_norm: positive, finite (the pages give no
+ * value).  out [4] device double.  A tensor listed twice is scaled twice.
+ * Same arguments, limits and workspace as sparseclip_norm otherwise; the
+ * tensors are writable device fp32, 16-byte aligned. */
+int32_t sparseclip_clip(float* const* dense, const int64_t* dense_len, int32_t n_dense,
+                        float* const* sparse, const int64_t* sparse_len, int32_t n_sparse,
+                        int32_t num_experts, double max_norm, double* out, void* workspace,
+                        size_t workspace_bytes, moe_stream_t stream);
 
 /* sparseclip_norm without a workspace, for callers that cannot allocate
  * device memory: a runtime whose HBM is handed out once at start-up by its

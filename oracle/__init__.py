@@ -55,6 +55,8 @@ def _load():
         "oracle_layer_forward": ([i64, i32, i32, i32, i32, i32, i32, i32, i32, u64] + [vp] * 19
                                  + [i32], None),
         "oracle_sparseclip_norm": ([vp, vp, i32, vp, vp, i32, i32], dbl),
+        "oracle_aux_loss": ([i64, i32, vp, dbl, vp, vp, vp], None),
+        "oracle_sparseclip_clip": ([vp, vp, i32, vp, vp, i32, i32, dbl, vp], dbl),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -226,3 +228,34 @@ def sparseclip_norm(dense, sparse, E):
                                                 ctypes.cast(dl, ctypes.c_void_p), len(dense),
                                                 ctypes.cast(sp, ctypes.c_void_p),
                                                 ctypes.cast(sl, ctypes.c_void_p), len(sparse), E))
+
+
+def aux_loss(logits, alpha=1e-2):
+    """Switch load-balancing loss (eqs. 4-6) and mean routing entropy from fp32
+    logits [T, E]: returns (loss, entropy, f [E], P [E]) in double."""
+    assert logits.dtype == torch.float32 and logits.is_contiguous()
+    T, E = logits.shape
+    out = torch.zeros(2, dtype=torch.float64)
+    f = torch.zeros(E, dtype=torch.float64)
+    P = torch.zeros(E, dtype=torch.float64)
+    _load().oracle_aux_loss(T, E, _p(logits), float(alpha), _p(out), _p(f), _p(P))
+    return float(out[0]), float(out[1]), f, P
+
+
+def sparseclip_clip(dense, sparse, E, max_norm):
+    """Clip lists of contiguous fp32 CPU tensors in place; returns (coef, norm)."""
+    def arr(ts):
+        ptrs = (ctypes.c_void_p * max(1, len(ts)))(*[t.data_ptr() for t in ts])
+        lens = (ctypes.c_int64 * max(1, len(ts)))(*[t.numel() for t in ts])
+        return ptrs, lens
+    for t in list(dense) + list(sparse):
+        assert t.dtype == torch.float32 and t.is_contiguous() and t.device.type == "cpu"
+    dp, dl = arr(dense)
+    sp, sl = arr(sparse)
+    norm = ctypes.c_double(0.0)
+    coef = _load().oracle_sparseclip_clip(ctypes.cast(dp, ctypes.c_void_p),
+                                          ctypes.cast(dl, ctypes.c_void_p), len(dense),
+                                          ctypes.cast(sp, ctypes.c_void_p),
+                                          ctypes.cast(sl, ctypes.c_void_p), len(sparse), E,
+                                          float(max_norm), ctypes.byref(norm))
+    return float(coef), float(norm.value)

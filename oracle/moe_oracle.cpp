@@ -14,7 +14,9 @@
 //     them); sec. 2.4 "selective precision": the router works in float32.
 //   * "[Paper review] TorchScale: Transformers at Scale", proposed method:
 //     X-MoE top-1 / top-2 routing; SparseClip ||g||_2 = ||(g_d, kappa g_s)||_2
-//     with kappa = 1/sqrt(E).
+//     with kappa = 1/sqrt(E); key results: the routing entropy it tracks.
+//   * Switch notes sec. 2.2, the differentiable load-balancing loss, eqs.
+//     (4)-(6).
 //   * "[Paper review] PanGu-Sigma", proposed method: Random Routed Experts —
 //     experts grouped by domain, each token sent uniformly at random to an
 //     expert of its domain's group through an unweighted gate.
@@ -353,6 +355,68 @@ double oracle_sparseclip_norm(const float* const* dense, const int64_t* dense_le
     for (int64_t i = 0; i < sparse_len[s]; ++i) ss += static_cast<double>(sparse[s][i]) * sparse[s][i];
   const double kappa = 1.0 / std::sqrt(static_cast<double>(E));
   return std::sqrt(sd + kappa * kappa * ss);
+}
+
+// TorchScale review, SparseClip as gradient clipping: every gradient (dense
+// and expert) is multiplied by coef = min(1, max_norm / ||g||_2), with the
+// reweighted norm of oracle_sparseclip_norm; each product is taken in double
+// and rounded once to fp32.  Tensors are updated in place.  Returns coef.
+double oracle_sparseclip_clip(float* const* dense, const int64_t* dense_len, int32_t n_dense,
+                              float* const* sparse, const int64_t* sparse_len, int32_t n_sparse,
+                              int32_t E, double max_norm, double* norm_out) {
+  const double norm = oracle_sparseclip_norm(dense, dense_len, n_dense, sparse, sparse_len,
+                                             n_sparse, E);
+  const double coef = norm > max_norm ? max_norm / norm : 1.0;
+  if (norm_out) *norm_out = norm;
+  for (int32_t s = 0; s < n_dense; ++s)
+    for (int64_t i = 0; i < dense_len[s]; ++i)
+      dense[s][i] = static_cast<float>(static_cast<double>(dense[s][i]) * coef);
+  for (int32_t s = 0; s < n_sparse; ++s)
+    for (int64_t i = 0; i < sparse_len[s]; ++i)
+      sparse[s][i] = static_cast<float>(static_cast<double>(sparse[s][i]) * coef);
+  return coef;
+}
+
+// Switch notes sec. 2.2, "A Differentiable Load Balancing Loss", eqs. (4)-(6):
+//   f_i = (1/T) #{tokens x : argmax p(x) = i}          (eq. 5)
+//   P_i = (1/T) sum_x p_i(x)                            (eq. 6, p from eq. 1)
+//   loss = alpha * N * sum_i f_i P_i   (N = E experts)  (eq. 4)
+// The argmax is taken on the fp32 logits with ties to the lower index (the
+// top-1 choice of oracle_gate_topk).  Also the routing entropy the TorchScale
+// review tracks, read as the mean over tokens of -sum_i p_i(x) ln p_i(x)
+// (terms with p_i = 0 contribute 0).  out[0] = loss, out[1] = entropy;
+// f, P (nullable) receive the two vectors.  All in double.
+void oracle_aux_loss(int64_t T, int32_t E, const float* logits, double alpha, double* out,
+                     double* f, double* P) {
+  std::vector<double> fs(E, 0.0), Ps(E, 0.0), p(E);
+  double ent = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    const float* h = logits + t * E;
+    int32_t best = 0;
+    for (int32_t e = 1; e < E; ++e)
+      if (h[e] > h[best]) best = e;  // strict: the lower index wins a tie
+    const double m = h[best];
+    double z = 0.0;
+    for (int32_t e = 0; e < E; ++e) z += std::exp(static_cast<double>(h[e]) - m);
+    double ht = 0.0;
+    for (int32_t e = 0; e < E; ++e) {
+      p[e] = std::exp(static_cast<double>(h[e]) - m) / z;
+      Ps[e] += p[e];
+      if (p[e] > 0.0) ht -= p[e] * std::log(p[e]);
+    }
+    fs[best] += 1.0;
+    ent += ht;
+  }
+  double dot = 0.0;
+  for (int32_t e = 0; e < E; ++e) {
+    fs[e] /= static_cast<double>(T);
+    Ps[e] /= static_cast<double>(T);
+    dot += fs[e] * Ps[e];
+    if (f) f[e] = fs[e];
+    if (P) P[e] = Ps[e];
+  }
+  out[0] = alpha * E * dot;
+  out[1] = ent / static_cast<double>(T);
 }
 
 }  // extern "C"

@@ -67,8 +67,11 @@ SIGNATURES = {
     "moe_combine": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "moe_layer_forward": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp],
                           _i32),
+    "moe_aux_workspace_size": ([_PCFG], _sz),
+    "moe_aux_loss": ([_PCFG, _vp, _dbl, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "sparseclip_norm": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "sparseclip_norm_noalloc": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
+    "sparseclip_clip": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _dbl, _vp, _vp, _sz, _vp], _i32),
 }
 
 
@@ -167,6 +170,26 @@ def router(cfg, x, Wr, bias=None, logits=None, status=None, stream=None):
                           _ptr(logits, "logits"), _ptr(status, "status"), _stream(stream)),
            "moe_router")
     return logits
+
+
+def aux_workspace_size(cfg: MoEConfig) -> int:
+    return int(lib.moe_aux_workspace_size(ctypes.byref(cfg)))
+
+
+def aux_loss(cfg, logits, alpha=1e-2, workspace=None, stream=None):
+    """Switch load-balancing loss and routing entropy from fp32 logits [T, E].
+
+    Returns device float64 tensors: out [2] (loss, entropy), f [E], P [E]."""
+    dev = logits.device
+    out = torch.empty(2, dtype=torch.float64, device=dev)
+    f = torch.empty(cfg.E, dtype=torch.float64, device=dev)
+    P = torch.empty(cfg.E, dtype=torch.float64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(256, aux_workspace_size(cfg)), dtype=torch.uint8, device=dev)
+    _check(lib.moe_aux_loss(ctypes.byref(cfg), _ptr(logits, "logits"), float(alpha),
+                            _ptr(out, "out"), _ptr(f, "f"), _ptr(P, "P"), _ptr(workspace, "workspace"),
+                            workspace.numel(), _stream(stream)), "moe_aux_loss")
+    return out, f, P
 
 
 def topk_assign(cfg, logits=None, domain_id=None, out=None, workspace=None, status=None,
@@ -322,4 +345,34 @@ def sparseclip_norm(dense, sparse, num_experts, out=None, workspace=None, stream
                                ctypes.cast(sp, _vp), ctypes.cast(sl, _vp), len(sparse),
                                num_experts, _ptr(out, "out"), _ptr(workspace, "workspace"),
                                workspace.numel(), _stream(stream)), "sparseclip_norm")
+    return out
+
+
+def sparseclip_clip(dense, sparse, num_experts, max_norm, out=None, workspace=None, stream=None):
+    """SparseClip clipping of lists of fp32 CUDA tensors, in place; returns
+    device double[4] = (norm before clipping, sum of squares dense, sum of
+    squares expert, coef applied)."""
+    dense, sparse = list(dense), list(sparse)
+    dev = (dense + sparse)[0].device
+    if out is None:
+        out = torch.empty(4, dtype=torch.float64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(16, sparseclip_workspace_size(len(dense), len(sparse))),
+                                dtype=torch.uint8, device=dev)
+
+    def arrays(ts, name):
+        ptrs = (ctypes.c_void_p * max(1, len(ts)))(*[_ptr(t, name) for t in ts])
+        lens = (ctypes.c_int64 * max(1, len(ts)))(*[t.numel() for t in ts])
+        return ptrs, lens
+
+    for t in dense + sparse:
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError("SparseClip gradients must be contiguous fp32")
+    dp, dl = arrays(dense, "dense")
+    sp, sl = arrays(sparse, "sparse")
+    _check(lib.sparseclip_clip(ctypes.cast(dp, _vp), ctypes.cast(dl, _vp), len(dense),
+                               ctypes.cast(sp, _vp), ctypes.cast(sl, _vp), len(sparse),
+                               num_experts, float(max_norm), _ptr(out, "out"),
+                               _ptr(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           "sparseclip_clip")
     return out

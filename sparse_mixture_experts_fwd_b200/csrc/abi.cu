@@ -282,6 +282,36 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert
   return launch_combine(*cfg, ye, expert_idx, gate, slot, kept, y, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t moe_aux_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return aux_workspace_bytes(*cfg);
+}
+
+int32_t moe_aux_loss(const moe_config* cfg, const float* logits, double alpha, double* out,
+                     double* f, double* P, void* workspace, size_t workspace_bytes,
+                     moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->mode != MOE_ROUTE_TOPK)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_aux_loss: RRE routing has no learned gate");
+  if (cfg->T > 0) MOE_TRY(need_ptr4(logits, "logits"));
+  auto need8 = [](const void* q, const char* name, bool required) -> int32_t {
+    if (!q) return required ? fail(MOE_ERR_INVALID_ARGUMENT, std::string(name) + " is null") : MOE_OK;
+    if (reinterpret_cast<uintptr_t>(q) & 7u)
+      return fail(MOE_ERR_ALIGNMENT, std::string(name) + " is not 8-byte aligned");
+    return MOE_OK;
+  };
+  MOE_TRY(need8(out, "out", true));
+  MOE_TRY(need8(f, "f", false));
+  MOE_TRY(need8(P, "P", false));
+  const size_t need = aux_workspace_bytes(*cfg);
+  if (!workspace || workspace_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "moe_aux_loss: workspace needs " + std::to_string(need) + " bytes");
+  MOE_TRY(need_ptr(workspace, "workspace"));
+  return launch_aux_loss(*cfg, logits, alpha, out, f, P, workspace,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
 int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
                           const int32_t* domain_id, const void* W1, const void* W2, void* y,
                           void* workspace, size_t workspace_bytes, int32_t* status,

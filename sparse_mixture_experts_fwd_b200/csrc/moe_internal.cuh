@@ -91,6 +91,10 @@ int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* exper
                         const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
                         unsigned int* zero_words = nullptr, int n_zero = 0,
                         void* y_zero = nullptr);
+// Switch load-balancing loss (eqs. 4-6) and routing entropy from logits [T, E]
+size_t aux_workspace_bytes(const moe_config& c);
+int32_t launch_aux_loss(const moe_config& c, const float* logits, double alpha, double* out,
+                        double* f, double* P, void* workspace, cudaStream_t s);
 int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* expert_idx,
                        const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
                        cudaStream_t s);

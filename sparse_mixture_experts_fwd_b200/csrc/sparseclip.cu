@@ -1,7 +1,9 @@
 // SparseClip global gradient norm ("[Paper review] TorchScale: Transformers
 // at Scale", proposed method):
 //   ||g||_2 = ||(g_d, kappa g_s)||_2 = sqrt(Sd + kappa^2 Ss),  kappa = 1/sqrt(E)
-// where Sd / Ss are the sums of squares of the dense / expert gradients.
+// where Sd / Ss are the sums of squares of the dense / expert gradients, and
+// the clipping step that uses it: every gradient scaled by
+// min(1, max_norm / ||g||_2).
 //
 // One bandwidth pass: a fixed grid of kGrid blocks streams every tensor with
 // 16-byte loads (4 in flight per thread), squares and sums each float4 in
@@ -54,7 +56,7 @@ __device__ __forceinline__ float sq4(const float4& v) {
 
 __global__ void __launch_bounds__(kBlock) sumsq_kernel(const ClipBatch b, double* partials) {
   __shared__ double s_red[kBlock / 32];
-  double acc[2] = {0.0, 0.0};
+  double acc_d = 0.0, acc_e = 0.0;  // dense, expert
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x;
   const int64_t nth = static_cast<int64_t>(gridDim.x) * kBlock;
   for (int s = 0; s < b.n; ++s) {
@@ -79,10 +81,10 @@ __global__ void __launch_bounds__(kBlock) sumsq_kernel(const ClipBatch b, double
       const float v = __ldg(p + j);
       a += static_cast<double>(v * v);
     }
-    acc[b.seg[s].cls] += a;
+    if (b.seg[s].cls) acc_e += a; else acc_d += a;
   }
-  const double d = block_sum(acc[0], s_red);
-  const double e = block_sum(acc[1], s_red);
+  const double d = block_sum(acc_d, s_red);
+  const double e = block_sum(acc_e, s_red);
   if (threadIdx.x == 0) {
     partials[2 * blockIdx.x] = d;
     partials[2 * blockIdx.x + 1] = e;
@@ -103,6 +105,51 @@ __global__ void __launch_bounds__(kBlock) finish_kernel(const double* partials, 
     out[0] = sqrt(sd + ss / static_cast<double>(num_experts));  // kappa^2 = 1/E
     out[1] = sd;
     out[2] = ss;
+  }
+}
+
+// Clipping step: every tensor (dense and expert) scaled in place by
+// coef = min(1, max_norm / norm), norm = out[0] written by finish_kernel on
+// the same stream.  When coef is 1 nothing is written.  Block 0 records coef
+// in out[3].  16-byte loads and stores, the same grid-stride order as the sum.
+struct ScaleSeg {
+  float* ptr;
+  int64_t len;
+};
+struct ScaleBatch {
+  ScaleSeg seg[kSegsPerLaunch];
+  int32_t n;
+};
+
+__global__ void __launch_bounds__(kBlock) scale_kernel(const ScaleBatch b, double max_norm,
+                                                       double* out, int write_coef) {
+  const double norm = out[0];
+  const double coefd = norm > max_norm ? max_norm / norm : 1.0;
+  if (write_coef && blockIdx.x == 0 && threadIdx.x == 0) out[3] = coefd;
+  if (coefd == 1.0) return;
+  const float c = static_cast<float>(coefd);
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x;
+  const int64_t nth = static_cast<int64_t>(gridDim.x) * kBlock;
+  for (int s = 0; s < b.n; ++s) {
+    float* p = b.seg[s].ptr;
+    const int64_t n = b.seg[s].len;
+    const int64_t n4 = n >> 2;
+    float4* p4 = reinterpret_cast<float4*>(p);
+    int64_t i = gtid;
+    for (; i + nth < n4; i += 2 * nth) {
+      float4 v0 = p4[i];
+      float4 v1 = p4[i + nth];
+      v0.x *= c; v0.y *= c; v0.z *= c; v0.w *= c;
+      v1.x *= c; v1.y *= c; v1.z *= c; v1.w *= c;
+      p4[i] = v0;
+      p4[i + nth] = v1;
+    }
+    for (; i < n4; i += nth) {
+      float4 v = p4[i];
+      v.x *= c; v.y *= c; v.z *= c; v.w *= c;
+      p4[i] = v;
+    }
+    for (int64_t j = 4 * n4 + gtid; j < n; j += nth) p[j] *= c;
   }
 }
 
@@ -165,6 +212,41 @@ extern "C" int32_t sparseclip_norm(const float* const* dense, const int64_t* den
   }
   finish_kernel<<<1, kBlock, 0, s>>>(partials, static_cast<int>(launches * kGrid), num_experts, out);
   return check_launch("finish_kernel");
+}
+
+extern "C" int32_t sparseclip_clip(float* const* dense, const int64_t* dense_len, int32_t n_dense,
+                                   float* const* sparse, const int64_t* sparse_len,
+                                   int32_t n_sparse, int32_t num_experts, double max_norm,
+                                   double* out, void* workspace, size_t workspace_bytes,
+                                   moe_stream_t stream) {
+  set_last_error("");
+  if (!(max_norm > 0.0) || !std::isfinite(max_norm))
+    return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_clip: max_norm must be positive and finite");
+  // the norm first (validates every argument), into out[0..2]
+  int32_t rc = sparseclip_norm(dense, dense_len, n_dense, sparse, sparse_len, n_sparse,
+                               num_experts, out, workspace, workspace_bytes, stream);
+  if (rc != MOE_OK) return rc;
+  std::vector<ScaleSeg> segs;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int32_t n = pass == 0 ? n_dense : n_sparse;
+    float* const* ptrs = pass == 0 ? dense : sparse;
+    const int64_t* lens = pass == 0 ? dense_len : sparse_len;
+    for (int32_t i = 0; i < n; ++i)
+      if (lens[i] > 0) segs.push_back(ScaleSeg{ptrs[i], lens[i]});
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t launches =
+      std::max<int64_t>(1, (static_cast<int64_t>(segs.size()) + kSegsPerLaunch - 1) / kSegsPerLaunch);
+  for (int64_t l = 0; l < launches; ++l) {
+    ScaleBatch b{};
+    const size_t first = static_cast<size_t>(l) * kSegsPerLaunch;
+    b.n = static_cast<int32_t>(std::min<size_t>(kSegsPerLaunch, segs.size() - std::min(first, segs.size())));
+    for (int32_t i = 0; i < b.n; ++i) b.seg[i] = segs[first + i];
+    scale_kernel<<<kGrid, kBlock, 0, s>>>(b, max_norm, out, l == 0 ? 1 : 0);
+    rc = check_launch("scale_kernel");
+    if (rc != MOE_OK) return rc;
+  }
+  return MOE_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -114,6 +114,16 @@ def test_calls_rejected_on_host(moe):
     assert moe.lib.sparseclip_norm(None, None, 0, None, None, 0, 0, p, p, 1 << 20, None) == -1
     assert moe.lib.sparseclip_workspace_size(1, 64) == 1024 * 2 * 8
     assert moe.lib.sparseclip_workspace_size(-1, 0) == 0
+    # aux loss: RRE has no learned gate, out is required and 8-byte aligned,
+    # the workspace must be moe_aux_workspace_size bytes
+    ws = moe.lib.moe_aux_workspace_size(ctypes.byref(c))
+    assert ws > 0 and ws % 256 == 0
+    rre = cfg(moe, mode="rre", num_groups=4)
+    assert moe.lib.moe_aux_loss(ctypes.byref(rre), p, 0.01, p, None, None, p, 1 << 30, None) == -2
+    assert moe.lib.moe_aux_loss(ctypes.byref(c), p, 0.01, None, None, None, p, ws, None) == -1
+    assert moe.lib.moe_aux_loss(ctypes.byref(c), p, 0.01, ctypes.c_void_p(4100), None, None, p, ws,
+                                None) == -3
+    assert moe.lib.moe_aux_loss(ctypes.byref(c), p, 0.01, p, None, None, p, ws - 1, None) == -4
 
 
 def test_library_refuses_cpu_tensors(moe):

@@ -446,6 +446,43 @@ def test_layer_zero_tokens(moe, cuda_device):
 
 
 # ---------------------------------------------------------------------------
+# Switch load-balancing loss (eqs. 4-6) and routing entropy
+# ---------------------------------------------------------------------------
+
+def _check_aux(moe, cfg, logits, alpha=1e-2):
+    out, f, P = moe.aux_loss(cfg, logits.to("cuda"), alpha)
+    torch.cuda.synchronize()
+    loss, ent, f_ref, P_ref = oracle.aux_loss(logits.cpu().contiguous(), alpha)
+    # the same fp32 logits and tie rule on both sides: f (token counts / T) is exact
+    assert torch.equal(f.cpu(), f_ref)
+    # fp32 softmax per token, double sums: relative 1e-5 (the gate tolerance)
+    assert torch.allclose(P.cpu(), P_ref, rtol=GATE_RTOL, atol=1e-12)
+    assert math.isclose(float(out[0]), loss, rel_tol=GATE_RTOL, abs_tol=1e-15)
+    assert math.isclose(float(out[1]), ent, rel_tol=GATE_RTOL, abs_tol=1e-6)
+
+
+def test_aux_loss_full(moe, cuda_device, case):
+    if case.w.mode != "topk":
+        pytest.skip("RRE has no learned gate")
+    _check_aux(moe, case.cfg, case.ref["logits"])
+
+
+@pytest.mark.parametrize("T,E", [(1, 1), (1, 8), (1000, 40), (4097, 256), (300, 7)])
+def test_aux_loss_shapes(moe, cuda_device, T, E):
+    cfg = moe.make_config(T, 64, 64, E, 1, 1, dtype=torch.float32)
+    _check_aux(moe, cfg, synth.normal(3, 2, (T, E), 2.0, torch.float32))
+    # equal logits: every argmax is expert 0 and the loss is exactly alpha
+    _check_aux(moe, cfg, torch.zeros(T, E))
+
+
+def test_aux_loss_zero_tokens(moe, cuda_device):
+    cfg = moe.make_config(0, 64, 64, 8, 1, 0, dtype=torch.float32)
+    out, f, P = moe.aux_loss(cfg, torch.zeros(1, 8, device="cuda"))
+    torch.cuda.synchronize()
+    assert out.tolist() == [0.0, 0.0] and float(f.abs().sum()) == 0 and float(P.abs().sum()) == 0
+
+
+# ---------------------------------------------------------------------------
 # a8 SparseClip norm
 # ---------------------------------------------------------------------------
 
@@ -477,3 +514,53 @@ def test_sparseclip_segments_and_tails(moe, cuda_device):
                               [torch.tensor([6.0, 8.0], device=dev)], 4)
     torch.cuda.synchronize()
     assert abs(out[0].item() - math.sqrt(50.0)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# SparseClip clipping step
+# ---------------------------------------------------------------------------
+
+def _clip_case(moe, dense, sparse, E, max_norm):
+    dev = "cuda"
+    gd = [t.to(dev) for t in dense]
+    gs = [t.to(dev) for t in sparse]
+    out = moe.sparseclip_clip(gd, gs, E, max_norm)
+    torch.cuda.synchronize()
+    rd = [t.clone() for t in dense]
+    rs = [t.clone() for t in sparse]
+    coef, norm = oracle.sparseclip_clip(rd, rs, E, max_norm)
+    got = out.cpu().tolist()
+    assert abs(got[0] - norm) <= GATE_RTOL * norm
+    # coef = max_norm / norm: the norm's relative error carries over
+    assert abs(got[3] - coef) <= GATE_RTOL * coef
+    if got[3] == 1.0:  # no clipping: nothing written
+        assert all(torch.equal(g.cpu(), t) for g, t in zip(gd + gs, dense + sparse))
+    for g, r in zip(gd + gs, rd + rs):
+        # fp32 product with fp32(coef) vs the exact product rounded once
+        tol = (abs(got[3] - coef) / coef + 2 ** -22) * r.abs() + 1e-30
+        assert bool(((g.cpu() - r).abs() <= tol).all())
+    return got
+
+
+def test_sparseclip_clip(moe, cuda_device):
+    dense = [synth.normal(2, 6, (n,), 1e-3, torch.float32) for n in (1, 3, 4097, 0, 1_000_003)]
+    sparse = [synth.normal(2, 7 + 16 * s, (513 + 7 * s,), 1e-3, torch.float32) for s in range(200)]
+    norm = oracle.sparseclip_norm(dense, sparse, 64)
+    got = _clip_case(moe, dense, sparse, 64, norm / 4)   # clips: every tensor scaled by ~1/4
+    assert got[3] == pytest.approx(0.25, rel=GATE_RTOL)
+    got = _clip_case(moe, dense, sparse, 64, norm * 4)   # no clipping: values bit-identical
+    assert got[3] == 1.0
+    # hand-worked example: coef 1/sqrt(2), clipped norm 5
+    gd = [torch.tensor([3.0, 4.0], device="cuda")]
+    gs = [torch.tensor([6.0, 8.0], device="cuda")]
+    out = moe.sparseclip_clip(gd, gs, 4, 5.0)
+    n2 = moe.sparseclip_norm(gd, gs, 4)
+    torch.cuda.synchronize()
+    assert abs(out[3].item() - 1 / math.sqrt(2.0)) < 1e-15
+    assert abs(n2[0].item() - 5.0) < 1e-6
+
+
+def test_sparseclip_clip_rejects(moe, cuda_device):
+    t = torch.zeros(8, device="cuda")
+    with pytest.raises(moe.MoEError):
+        moe.sparseclip_clip([t], [t.clone()], 4, 0.0)

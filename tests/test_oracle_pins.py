@@ -338,3 +338,101 @@ def test_sparseclip_special_cases(oracle_lib):
     # E = 64: kappa^2 = 1/64 exactly
     sn = float(np.linalg.norm(np.concatenate([t.double().numpy() for t in gs])))
     assert oracle.sparseclip_norm(gd, gs, 64) == pytest.approx(math.sqrt(dn ** 2 + sn ** 2 / 64), rel=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Switch load-balancing loss (eqs. 4-6) and routing entropy
+# ---------------------------------------------------------------------------
+
+def test_aux_loss_hand_examples(oracle_lib):
+    g = read_golden("aux_loss_example.txt")
+    alpha = float(g["alpha"][0][0])
+    for case in ("caseA", "caseB"):
+        lg = torch.tensor([[float(v) * math.log(3.0) for v in row] for row in g[case + "_l3"]],
+                          dtype=torch.float32)
+        loss, ent, f, P = oracle.aux_loss(lg, alpha)
+        # ln 3 is rounded to fp32 in the logits: |rel err| ~ 1e-7
+        assert loss == pytest.approx(float(g[case + "_loss"][0][0]), rel=1e-6)
+        assert ent == pytest.approx(float(g[case + "_entropy"][0][0]), rel=1e-6)
+        assert f.tolist() == [float(v) for v in g[case + "_f"][0]]
+        assert P.tolist() == pytest.approx([float(v) for v in g[case + "_P"][0]], rel=1e-6)
+
+
+@pytest.mark.parametrize("E", [1, 3, 8, 64, 256])
+def test_aux_loss_closed_forms(oracle_lib, E):
+    alpha = 1e-2
+    # equal logits: p uniform (P_i = 1/E, entropy ln E); every argmax is expert 0
+    # (tie -> lower index), so f = e_0 and the loss is alpha * E * (1/E) = alpha
+    loss, ent, f, P = oracle.aux_loss(torch.zeros(7, E), alpha)
+    assert loss == pytest.approx(alpha, rel=1e-12)
+    assert ent == pytest.approx(math.log(E), abs=1e-12)
+    assert f[0] == 1.0 and float(f.sum()) == 1.0
+    assert torch.allclose(P, torch.full((E,), 1.0 / E, dtype=torch.float64), rtol=1e-12)
+    # a balanced assignment (token t peaks at expert t mod E, n tokens per expert):
+    # f_i = P_i = 1/E by symmetry, so the loss is alpha (the minimum the notes
+    # describe); each token's entropy is ln(e^L + E - 1) - L e^L / (e^L + E - 1)
+    L, n = 3.0, 5
+    lg = torch.zeros(n * E, E)
+    lg[torch.arange(n * E), torch.arange(n * E) % E] = L
+    loss, ent, f, P = oracle.aux_loss(lg, alpha)
+    z = math.exp(L) + E - 1
+    assert loss == pytest.approx(alpha, rel=1e-12)
+    assert ent == pytest.approx(math.log(z) - L * math.exp(L) / z, rel=1e-12, abs=1e-15)
+    assert torch.allclose(f, torch.full((E,), 1.0 / E, dtype=torch.float64), rtol=1e-12)
+    assert torch.allclose(P, torch.full((E,), 1.0 / E, dtype=torch.float64), rtol=1e-12)
+
+
+def test_aux_loss_against_library_softmax(oracle_lib):
+    # an independent statement of eqs. (4)-(6) with library routines
+    T, E, alpha = 513, 40, 1e-2
+    lg = synth.normal(5, 2, (T, E), 1.5, torch.float32)
+    loss, ent, f, P = oracle.aux_loss(lg, alpha)
+    p = torch.softmax(lg.double(), dim=1)
+    P_ref = p.mean(0)
+    f_ref = torch.bincount(lg.argmax(1), minlength=E).double() / T  # continuous draws: no ties
+    assert torch.allclose(P, P_ref, rtol=1e-12, atol=0)
+    assert torch.equal(f, f_ref)
+    assert loss == pytest.approx(alpha * E * float((f_ref * P_ref).sum()), rel=1e-12)
+    assert ent == pytest.approx(float(-(p * p.log()).sum(1).mean()), rel=1e-12)
+
+
+def test_sparseclip_clip_hand_example(oracle_lib):
+    g = read_golden("sparseclip_example.txt")
+    E = int(g["E"][0][0])
+    gd = torch.tensor([float(v) for v in g["g_dense"][0]])
+    gs = torch.tensor([float(v) for v in g["g_sparse"][0]])
+    d0, s0 = gd.clone(), gs.clone()
+    coef, norm = oracle.sparseclip_clip([gd], [gs], E, float(g["max_norm"][0][0]))
+    assert coef == pytest.approx(float(g["coef"][0][0]), rel=1e-15)
+    assert norm == pytest.approx(float(g["norm"][0][0]), rel=1e-15)
+    r = 1 / math.sqrt(2.0)
+    assert gd.tolist() == [float(torch.tensor(v * r, dtype=torch.float32)) for v in d0.tolist()]
+    assert gs.tolist() == [float(torch.tensor(v * r, dtype=torch.float32)) for v in s0.tolist()]
+    # after clipping the reweighted norm is max_norm (up to the fp32 rounding of the values)
+    assert oracle.sparseclip_norm([gd], [gs], E) == pytest.approx(5.0, rel=1e-7)
+
+
+def test_sparseclip_clip_special_cases(oracle_lib):
+    gd = [synth.normal(11, 6, (1001,), 1e-3, torch.float32)]
+    gs = [synth.normal(11, 7 + 16 * s, (503,), 1e-3, torch.float32) for s in range(4)]
+    norm = oracle.sparseclip_norm(gd, gs, 4)
+    # a threshold above the norm leaves every value untouched, bit for bit
+    before = [t.clone() for t in gd + gs]
+    coef, _ = oracle.sparseclip_clip(gd, gs, 4, 2 * norm)
+    assert coef == 1.0 and all(torch.equal(a, b) for a, b in zip(before, gd + gs))
+    # below it: every tensor scaled by the same max_norm / norm, the new norm is max_norm
+    coef, n2 = oracle.sparseclip_clip(gd, gs, 4, norm / 3)
+    assert n2 == pytest.approx(norm, rel=1e-15) and coef == pytest.approx(1 / 3, rel=1e-12)
+    for a, b in zip(before, gd + gs):
+        assert torch.allclose(b.double(), a.double() / 3, rtol=2 ** -23, atol=0)
+    assert oracle.sparseclip_norm(gd, gs, 4) == pytest.approx(norm / 3, rel=1e-6)
+    # E = 1 (kappa = 1): the same coefficient as the library's clip-by-global-norm
+    # (which adds 1e-6 to the norm)
+    t = [synth.normal(12, 6, (777,), 1.0, torch.float32), synth.normal(12, 8, (333,), 1.0, torch.float32)]
+    lib_t = [x.clone().requires_grad_(True) for x in t]
+    for x in lib_t:
+        x.grad = x.detach().clone()
+    torch.nn.utils.clip_grad_norm_(lib_t, max_norm=1.0)
+    oracle.sparseclip_clip([t[0]], [t[1]], 1, 1.0)
+    for a, x in zip(t, lib_t):
+        assert torch.allclose(a, x.grad, rtol=1e-5, atol=0)
