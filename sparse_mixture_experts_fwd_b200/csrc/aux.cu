@@ -12,7 +12,7 @@
 // and the softmax sum by shuffles; each lane accumulates p for its experts
 // in double across the warp's tokens, the argmax is counted in shared
 // memory, H(p) = ln(s) - sum_e p_e (h_e - m) per token.  Each block (at most
-// two per SM) writes its partial P[E], counts[E] and entropy sum.  Pass 2: a
+// four per SM) writes its partial P[E], counts[E] and entropy sum.  Pass 2: a
 // block per expert adds that expert's partials (strided, then a fixed tree:
 // deterministic).  Pass 3 (one block): sum_e f_e P_e and the entropy.
 #include <climits>
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(256) aux_final_kernel(int64_t T, int E, int nb
 
 int aux_blocks(const moe_config& c) {
   const int64_t want = (c.T + kAuxWarps * 4 - 1) / (kAuxWarps * 4);  // >= 4 tokens per warp
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 2;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 4;  // 4 blocks of 256 per SM fit
   return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
