@@ -18,6 +18,7 @@ REGIMES = [
     ("xmoe_top2", {"T": 4096, "d_model": 256, "d_ff": 512}),            # top-2, C = 128
     ("xmoe_top2", {"T": 8192, "d_model": 256, "d_ff": 512}),            # C = 256
     ("pangu_rre", {"T": 26215, "d_model": 256, "d_ff": 512}),           # RRE, C = 512
+    ("pangu_rre", {"T": 32768, "d_model": 256, "d_ff": 512}),           # C = 640
 ]
 
 

@@ -200,6 +200,8 @@ FFN_SHAPES = {
     "sm_pairs": (6, 512, 256, 512, [512, 0, 257, 256, 1, 300]),
     # C >= 512, three 256-row blocks (the last ragged) and a 2048-deep K loop in GEMM 2
     "sm_pairs_long_k": (3, 600, 512, 2048, [600, 0, 513]),
+    # C > 512: last 256-row blocks holding 188, 100 (the only block), 128 and 89 rows
+    "sm_pairs_tails": (5, 700, 256, 512, [700, 100, 0, 640, 601]),
     # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
     "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
 }
