@@ -45,7 +45,7 @@ extern "C" {
 
 typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 enum moe_error {
   MOE_OK = 0,
@@ -58,12 +58,18 @@ enum moe_error {
 
 enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 };
 enum moe_route_mode { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RRE = 1 };
+/* Expert network.  RELU: H = ReLU(x W1^T), out = H W2^T, W1 [E, f, d].
+ * GEGLU (a gated linear unit in the feed-forward layer, "MosaicBERT" page:
+ * the FFN uses GLU): W1 [E, 2f, d] whose rows 2i and 2i+1 are the gate and the
+ * linear projection of hidden unit i, H_i = GELU(x . W1[2i]) * (x . W1[2i+1])
+ * with GELU(a) = a * Phi(a) (the erf form), out = H W2^T; bf16 layers only. */
+enum moe_expert { MOE_EXPERT_RELU = 0, MOE_EXPERT_GEGLU = 1 };
 enum moe_status_bits {
   MOE_STATUS_TIMEOUT = 1,   /* a pipeline wait gave up after 1 s; outputs invalid     */
   MOE_STATUS_BAD_DOMAIN = 2 /* an RRE domain id was outside 0..G-1 (routed as 0)       */
 };
 
-/* One MoE layer.  48 bytes, no padding. */
+/* One MoE layer.  56 bytes, no padding. */
 typedef struct moe_config {
   int64_t T;          /* tokens in the batch (>= 0)                                    */
   int32_t d_model;    /* token width d                                                 */
@@ -74,6 +80,8 @@ typedef struct moe_config {
   int32_t mode;       /* enum moe_route_mode                                           */
   int32_t num_groups; /* RRE: G domain groups, E % G == 0; ignored for TOPK            */
   int32_t dtype;      /* enum moe_dtype of x, W_r, W1, W2, xe, H, ye, y                */
+  int32_t expert;     /* enum moe_expert (0 = ReLU FFN)                                 */
+  int32_t reserved;   /* must be 0                                                      */
   uint64_t seed;      /* RRE: seed of the splitmix64 routing hash; ignored for TOPK    */
 } moe_config;
 
@@ -175,6 +183,8 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert
 /* Expert FFNs as one grouped computation over the kept rows:
  *   H[e, r, :]  = round(ReLU(xe[e, r, :] . W1[e]^T))   W1 [E, f, d]
  *   ye[e, r, :] = round(H[e, r, :] . W2[e]^T)          W2 [E, d, f]
+ * (cfg->expert == MOE_EXPERT_GEGLU: W1 [E, 2f, d] and H[e, r, i] =
+ * round(GELU(xe[e, r, :] . W1[e, 2i]) * (xe[e, r, :] . W1[e, 2i + 1])))
  * for r < kept_cnt[e] (device int32 [E], values in 0..C).  xe, ye
  * [E, C, d] and H [E, C, f] (caller-provided scratch) in cfg->dtype; other
  * rows of H and ye are left untouched.  bf16: one persistent tcgen05 kernel

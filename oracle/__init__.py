@@ -49,11 +49,12 @@ def _load():
         "oracle_assign": ([i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp], None),
         "oracle_dispatch": ([i64, i32, i32, i32, i32, vp, vp, vp, vp], None),
         "oracle_expert_row": ([i32, i32, i32, vp, vp, vp, vp, vp], None),
-        "oracle_expert_ffn": ([i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32], None),
+        "oracle_expert_row_geglu": ([i32, i32, i32, vp, vp, vp, vp, vp], None),
+        "oracle_expert_ffn": ([i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, i32], None),
         "oracle_combine": ([i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], None),
-        "oracle_token_forward": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp], None),
+        "oracle_token_forward": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, i32], None),
         "oracle_layer_forward": ([i64, i32, i32, i32, i32, i32, i32, i32, i32, u64] + [vp] * 19
-                                 + [i32], None),
+                                 + [i32, i32], None),
         "oracle_sparseclip_norm": ([vp, vp, i32, vp, vp, i32, i32], dbl),
         "oracle_aux_loss": ([i64, i32, vp, dbl, vp, vp, vp], None),
         "oracle_sparseclip_clip": ([vp, vp, i32, vp, vp, i32, i32, dbl, vp], dbl),
@@ -144,22 +145,27 @@ def dispatch(x, tok_of_row, kept_cnt, E, C):
     return xe.view(E, C, d)
 
 
-def expert_row(x_row, W1_e, W2_e, with_H=False):
-    f, d = W1_e.shape
+KINDS = {"relu": 0, "geglu": 1}
+
+
+def expert_row(x_row, W1_e, W2_e, with_H=False, kind="relu"):
+    """One token through one expert; kind "geglu" takes W1_e [2f, d] (gate, linear rows)."""
+    d = W1_e.shape[1]
+    f = W2_e.shape[1]
     out = torch.empty(d, dtype=x_row.dtype)
     H = torch.empty(f, dtype=x_row.dtype) if with_H else None
-    _load().oracle_expert_row(d, f, _dt(x_row), _p(x_row.contiguous()), _p(W1_e), _p(W2_e),
-                              _p(out), _p(H))
+    fn = _load().oracle_expert_row_geglu if kind == "geglu" else _load().oracle_expert_row
+    fn(d, f, _dt(x_row), _p(x_row.contiguous()), _p(W1_e), _p(W2_e), _p(out), _p(H))
     return (out, H) if with_H else out
 
 
-def expert_ffn(xe, W1, W2, kept_cnt, with_H=False, nthreads=None):
+def expert_ffn(xe, W1, W2, kept_cnt, with_H=False, nthreads=None, kind="relu"):
     E, C, d = xe.shape
-    f = W1.shape[1]
+    f = W2.shape[2]
     ye = torch.zeros(E, C, d, dtype=xe.dtype)
     H = torch.zeros(E, C, f, dtype=xe.dtype) if with_H else None
     _load().oracle_expert_ffn(d, f, E, C, _dt(xe), _p(xe), _p(W1), _p(W2), _p(kept_cnt), _p(H),
-                              _p(ye), nthreads or threads())
+                              _p(ye), nthreads or threads(), KINDS[kind])
     return (ye, H) if with_H else ye
 
 
@@ -172,22 +178,23 @@ def combine(ye, expert_idx, gate, slot, kept, T):
     return y
 
 
-def token_forward(x_row, W1, W2, expert_idx_row, gate_row, kept_row):
-    """Layer output of one token (eq. (2) for a single x) from full W1 [E,f,d], W2 [E,d,f]."""
-    E, f, d = W1.shape
+def token_forward(x_row, W1, W2, expert_idx_row, gate_row, kept_row, kind="relu"):
+    """Layer output of one token (eq. (2) for a single x) from full W1 [E,f,d] ([E,2f,d]
+    for GEGLU), W2 [E,d,f]."""
+    E, d, f = W2.shape
     k = expert_idx_row.numel()
     y = torch.empty(d, dtype=x_row.dtype)
     _load().oracle_token_forward(d, f, k, _dt(x_row), _p(x_row.contiguous()), _p(W1), _p(W2),
                                  _p(expert_idx_row.contiguous()), _p(gate_row.contiguous()),
-                                 _p(kept_row.contiguous()), _p(y))
+                                 _p(kept_row.contiguous()), _p(y), KINDS[kind])
     return y
 
 
 def layer_forward(x, W1, W2, *, E, k, C, Wr=None, bias=None, domain=None, G=1, seed=0,
-                  with_H=False, nthreads=None):
+                  with_H=False, nthreads=None, kind="relu"):
     """Every step of the layer; returns a dict of all intermediate results."""
     T, d = x.shape
-    f = W1.shape[1]
+    f = W2.shape[2]
     mode = 0 if domain is None else 1
     dt = x.dtype
     r = dict(
@@ -209,7 +216,7 @@ def layer_forward(x, W1, W2, *, E, k, C, Wr=None, bias=None, domain=None, G=1, s
         T, d, f, E, k, C, _dt(x), mode, G, seed, _p(x), _p(Wr), _p(bias), _p(domain), _p(W1),
         _p(W2), _p(r["logits"]), _p(r["expert_idx"]), _p(r["gate"]), _p(r["slot"]), _p(r["kept"]),
         _p(r["tok_of_row"]), _p(r["arrivals"]), _p(r["kept_cnt"]), _p(nd), _p(r["xe"]),
-        _p(r["H"]), _p(r["ye"]), _p(r["y"]), nthreads or threads())
+        _p(r["H"]), _p(r["ye"]), _p(r["y"]), nthreads or threads(), KINDS[kind])
     r["n_dropped"] = int(nd.item())
     return r
 

@@ -33,6 +33,9 @@
 //     double and rounds once;
 //   * RRE: group g owns experts [g*E/G, (g+1)*E/G); the in-group index is
 //     splitmix64(seed, t) mod (E/G), gate 1.
+//   * GLU experts ("MosaicBERT" page: GLU in the feed-forward layer, no
+//     formula): the GEGLU form, GELU(x W_gate) * (x W_linear), erf GELU, no
+//     biases, W1 rows interleaved (gate of unit i in row 2i, linear in 2i+1).
 //
 // Arithmetic: every product and sum is in double; values are rounded to the
 // activation type only at the points named above.
@@ -261,9 +264,43 @@ void oracle_expert_row(int32_t d, int32_t f, int32_t dtype, const void* x_row, c
 
 // All experts over their kept rows: ye[e, r] = E_e(xe[e, r]) for r < kept_cnt[e].
 // W1 is [E, f, d], W2 is [E, d, f].  H (nullable) is [E, C, f].
+// Gated linear unit in the feed-forward layer ("MosaicBERT" page: the FFN
+// uses GLU), GEGLU form: W1 [2f, d] holds, for hidden unit i, the gate
+// projection in row 2i and the linear projection in row 2i+1;
+//   H_i = GELU(x . W1[2i]) * (x . W1[2i+1]),  GELU(a) = a * Phi(a) = a (1 + erf(a / sqrt 2)) / 2,
+// in double, rounded once to the activation type; out = H . W2^T as for ReLU.
+void oracle_expert_row_geglu(int32_t d, int32_t f, int32_t dtype, const void* x_row,
+                             const void* W1, const void* W2, void* out_row, void* H_out) {
+  std::vector<double> H(f);
+  std::vector<uint32_t> hbuf(f);
+  void* hdst = H_out ? H_out : static_cast<void*>(hbuf.data());
+  for (int32_t i = 0; i < f; ++i) {
+    double g = 0.0, l = 0.0;
+    for (int32_t c = 0; c < d; ++c) {
+      const double xv = load(x_row, c, dtype);
+      g += xv * load(W1, static_cast<int64_t>(2 * i) * d + c, dtype);
+      l += xv * load(W1, static_cast<int64_t>(2 * i + 1) * d + c, dtype);
+    }
+    const double gelu = 0.5 * g * (1.0 + std::erf(g / std::sqrt(2.0)));
+    H[i] = store(hdst, i, dtype, gelu * l);
+  }
+  for (int32_t c = 0; c < d; ++c) {
+    double o = 0.0;
+    for (int32_t n = 0; n < f; ++n) o += H[n] * load(W2, static_cast<int64_t>(c) * f + n, dtype);
+    store(out_row, c, dtype, o);
+  }
+}
+
+// expert network by kind: 0 = ReLU FFN (W1 [f, d]), 1 = GEGLU (W1 [2f, d])
+static void expert_row_kind(int32_t kind, int32_t d, int32_t f, int32_t dtype, const void* x_row,
+                            const void* W1, const void* W2, void* out_row, void* H_out) {
+  if (kind == 1) oracle_expert_row_geglu(d, f, dtype, x_row, W1, W2, out_row, H_out);
+  else oracle_expert_row(d, f, dtype, x_row, W1, W2, out_row, H_out);
+}
+
 void oracle_expert_ffn(int32_t d, int32_t f, int32_t E, int32_t C, int32_t dtype, const void* xe,
                        const void* W1, const void* W2, const int32_t* kept_cnt, void* H, void* ye,
-                       int32_t threads) {
+                       int32_t threads, int32_t kind) {
   const size_t es = dtype == DT_BF16 ? 2 : 4;
   std::vector<int64_t> rows;
   for (int32_t e = 0; e < E; ++e)
@@ -271,8 +308,8 @@ void oracle_expert_ffn(int32_t d, int32_t f, int32_t E, int32_t C, int32_t dtype
   parallel_for(static_cast<int64_t>(rows.size()), threads, [&](int64_t i) {
     int64_t row = rows[i];
     int64_t e = row / C;
-    oracle_expert_row(d, f, dtype, static_cast<const char*>(xe) + row * d * es,
-                      static_cast<const char*>(W1) + e * f * d * es,
+    expert_row_kind(kind, d, f, dtype, static_cast<const char*>(xe) + row * d * es,
+                      static_cast<const char*>(W1) + e * (kind == 1 ? 2 : 1) * f * d * es,
                       static_cast<const char*>(W2) + e * d * f * es,
                       static_cast<char*>(ye) + row * d * es,
                       H ? static_cast<char*>(H) + row * f * es : nullptr);
@@ -303,15 +340,17 @@ void oracle_combine(int64_t T, int32_t d, int32_t k, int32_t C, int32_t dtype, c
 // W2 [E, d, f] are the full weight tensors.
 void oracle_token_forward(int32_t d, int32_t f, int32_t k, int32_t dtype, const void* x_row,
                           const void* W1, const void* W2, const int32_t* expert_idx_row,
-                          const float* gate_row, const uint8_t* kept_row, void* y_row) {
+                          const float* gate_row, const uint8_t* kept_row, void* y_row,
+                          int32_t kind) {
   const size_t es = dtype == DT_BF16 ? 2 : 4;
   std::vector<double> acc(d, 0.0);
   std::vector<uint32_t> out(d);  // room for d fp32 or bf16 values
   for (int32_t j = 0; j < k; ++j) {
     if (!kept_row[j]) continue;
     const int64_t e = expert_idx_row[j];
-    oracle_expert_row(d, f, dtype, x_row, static_cast<const char*>(W1) + e * f * d * es,
-                      static_cast<const char*>(W2) + e * d * f * es, out.data(), nullptr);
+    expert_row_kind(kind, d, f, dtype, x_row,
+                    static_cast<const char*>(W1) + e * (kind == 1 ? 2 : 1) * f * d * es,
+                    static_cast<const char*>(W2) + e * d * f * es, out.data(), nullptr);
     for (int32_t c = 0; c < d; ++c)
       acc[c] += static_cast<double>(gate_row[j]) * load(out.data(), c, dtype);
   }
@@ -329,7 +368,7 @@ void oracle_layer_forward(int64_t T, int32_t d, int32_t f, int32_t E, int32_t k,
                           const void* W1, const void* W2, float* logits, int32_t* expert_idx,
                           float* gate, int32_t* slot, uint8_t* kept, int32_t* tok_of_row,
                           int32_t* arrivals, int32_t* kept_cnt, int64_t* n_dropped, void* xe,
-                          void* H, void* ye, void* y, int32_t threads) {
+                          void* H, void* ye, void* y, int32_t threads, int32_t kind) {
   if (mode == 0) {
     oracle_router(T, d, E, dtype, x, Wr, bias, logits, threads);
     oracle_gate_topk(T, E, k, logits, expert_idx, gate, nullptr);
@@ -338,7 +377,7 @@ void oracle_layer_forward(int64_t T, int32_t d, int32_t f, int32_t E, int32_t k,
   }
   oracle_assign(T, E, k, C, expert_idx, slot, kept, tok_of_row, arrivals, kept_cnt, n_dropped);
   oracle_dispatch(T, d, E, C, dtype, x, tok_of_row, kept_cnt, xe);
-  oracle_expert_ffn(d, f, E, C, dtype, xe, W1, W2, kept_cnt, H, ye, threads);
+  oracle_expert_ffn(d, f, E, C, dtype, xe, W1, W2, kept_cnt, H, ye, threads, kind);
   oracle_combine(T, d, k, C, dtype, ye, expert_idx, gate, slot, kept, y);
 }
 

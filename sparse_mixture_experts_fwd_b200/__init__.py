@@ -31,10 +31,10 @@ _i32, _i64, _u64, _sz, _vp, _dbl = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uin
 
 
 class MoEConfig(ctypes.Structure):
-    """Mirror of ``moe_config`` (48 bytes)."""
+    """Mirror of ``moe_config`` (56 bytes)."""
     _fields_ = [("T", _i64), ("d_model", _i32), ("d_ff", _i32), ("E", _i32), ("k", _i32),
                 ("capacity", _i32), ("mode", _i32), ("num_groups", _i32), ("dtype", _i32),
-                ("seed", _u64)]
+                ("expert", _i32), ("reserved", _i32), ("seed", _u64)]
 
 
 class WorkspaceMap(ctypes.Structure):
@@ -133,11 +133,15 @@ def capacity(T: int, E: int, capacity_factor: float) -> int:
     return int(lib.moe_capacity(T, E, capacity_factor))
 
 
+EXPERTS = {"relu": 0, "geglu": 1}
+
+
 def make_config(T, d_model, d_ff, E, k, capacity_, *, dtype=torch.bfloat16, mode="topk",
-                num_groups=1, seed=0) -> MoEConfig:
+                num_groups=1, seed=0, expert="relu") -> MoEConfig:
+    """expert: "relu" (W1 [E, f, d]) or "geglu" (W1 [E, 2f, d], bf16 only)."""
     return MoEConfig(T=T, d_model=d_model, d_ff=d_ff, E=E, k=k, capacity=capacity_,
                      mode=ROUTE_TOPK if mode == "topk" else ROUTE_RRE, num_groups=num_groups,
-                     dtype=_dtype_code(dtype), seed=seed)
+                     dtype=_dtype_code(dtype), expert=EXPERTS[expert], reserved=0, seed=seed)
 
 
 def config_check(cfg: MoEConfig):

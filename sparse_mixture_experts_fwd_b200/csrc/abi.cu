@@ -62,6 +62,11 @@ int32_t check_cfg(const moe_config* c) {
     if (c->num_groups < 1 || c->E % c->num_groups != 0)
       return fail(MOE_ERR_INVALID_ARGUMENT, "RRE needs num_groups >= 1 dividing E");
   }
+  if (c->expert != MOE_EXPERT_RELU && c->expert != MOE_EXPERT_GEGLU)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "unknown expert network");
+  if (c->reserved != 0) return fail(MOE_ERR_INVALID_ARGUMENT, "reserved field must be 0");
+  if (c->expert == MOE_EXPERT_GEGLU && c->dtype != MOE_DTYPE_BF16)
+    return fail(MOE_ERR_UNSUPPORTED, "GEGLU experts are bf16 only");
   if (c->d_model < 1 || c->d_ff < 1) return fail(MOE_ERR_INVALID_ARGUMENT, "d_model/d_ff < 1");
   if (c->dtype == MOE_DTYPE_BF16) {
     if (c->d_model % 64 || c->d_ff % 64)
@@ -71,7 +76,7 @@ int32_t check_cfg(const moe_config* c) {
       return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d_model and d_ff multiples of 4");
   }
   const int64_t EC = int64_t(c->E) * c->capacity;
-  if (EC > kI32Max || int64_t(c->E) * c->d_ff > kI32Max || int64_t(c->E) * c->d_model > kI32Max)
+  if (EC > kI32Max || int64_t(c->E) * c->d_ff * 2 > kI32Max || int64_t(c->E) * c->d_model > kI32Max)
     return fail(MOE_ERR_UNSUPPORTED, "E*C, E*d_ff or E*d_model exceeds 2^31-1 rows");
   return MOE_OK;
 }

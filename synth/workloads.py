@@ -47,6 +47,7 @@ class Workload:
     capacity_factor: float
     dtype: str  # "f32" or "bf16": activations and weights
     mode: str = "topk"  # "topk" (softmax gate + top-k) or "rre"
+    expert: str = "relu"  # "relu" FFN (W1 [E, f, d]) or "geglu" (W1 [E, 2f, d])
     num_groups: int = 1
     hot_experts: int = 0
     hot_bias: float = 0.0
@@ -113,7 +114,8 @@ def layer_inputs(w: Workload, *, weights: bool = True, x_seed_offset: int = 0,
         out["domain"] = uniform_int(w.seed + x_seed_offset, TAGS["domain"], w.T, w.num_groups,
                                     threads=threads)
     if weights:
-        out["W1"] = normal(w.seed, TAGS["W1"], (w.E, w.d_ff, w.d_model), w.expert_std, dt,
+        rows = 2 * w.d_ff if w.expert == "geglu" else w.d_ff  # GEGLU: gate, linear rows
+        out["W1"] = normal(w.seed, TAGS["W1"], (w.E, rows, w.d_model), w.expert_std, dt,
                            threads=threads)
         out["W2"] = normal(w.seed, TAGS["W2"], (w.E, w.d_model, w.d_ff), w.expert_std, dt,
                            threads=threads)
@@ -122,11 +124,12 @@ def layer_inputs(w: Workload, *, weights: bool = True, x_seed_offset: int = 0,
 
 def expert_weights(w: Workload, e: int, threads: int | None = None):
     """W1[e] and W2[e] alone, generated from their offsets in the full streams."""
-    n1 = w.d_ff * w.d_model
-    W1 = normal(w.seed, TAGS["W1"], (w.d_ff, w.d_model), w.expert_std, w.torch_dtype,
+    rows = 2 * w.d_ff if w.expert == "geglu" else w.d_ff
+    n1, n2 = rows * w.d_model, w.d_ff * w.d_model
+    W1 = normal(w.seed, TAGS["W1"], (rows, w.d_model), w.expert_std, w.torch_dtype,
                 first=e * n1, threads=threads)
     W2 = normal(w.seed, TAGS["W2"], (w.d_model, w.d_ff), w.expert_std, w.torch_dtype,
-                first=e * n1, threads=threads)
+                first=e * n2, threads=threads)
     return W1, W2
 
 

@@ -35,8 +35,8 @@ def test_every_declared_symbol_is_exported(moe):
 
 
 def test_struct_layout(moe):
-    assert moe.lib.moe_abi_version() == 1
-    assert moe.lib.moe_config_size() == 48 == ctypes.sizeof(moe.MoEConfig)
+    assert moe.lib.moe_abi_version() == 2
+    assert moe.lib.moe_config_size() == 56 == ctypes.sizeof(moe.MoEConfig)
     assert moe.lib.moe_workspace_map_size() == ctypes.sizeof(moe.WorkspaceMap)
 
 
@@ -55,6 +55,7 @@ def cfg(moe, **kw):
     base.update(kw)
     import torch
     dtype = base.pop("dtype", torch.bfloat16)
+    dtype = torch.float32 if dtype == "f32" else dtype
     return moe.make_config(base.pop("T"), base.pop("d_model"), base.pop("d_ff"), base.pop("E"),
                            base.pop("k"), base.pop("capacity_"), dtype=dtype, **base)
 
@@ -63,7 +64,7 @@ def cfg(moe, **kw):
     (dict(E=0), -1), (dict(E=512), -2), (dict(k=3), -2), (dict(k=2, E=1), -1),
     (dict(capacity_=-1), -1), (dict(d_model=100), -2), (dict(d_ff=96), -2),
     (dict(mode="rre", k=2, num_groups=8), -1), (dict(mode="rre", num_groups=3), -1),
-    (dict(T=-5), -1),
+    (dict(T=-5), -1), (dict(expert="geglu", dtype="f32"), -2),
 ])
 def test_config_rejections(moe, kw, code):
     c = cfg(moe, **kw)

@@ -436,3 +436,67 @@ def test_sparseclip_clip_special_cases(oracle_lib):
     oracle.sparseclip_clip([t[0]], [t[1]], 1, 1.0)
     for a, x in zip(t, lib_t):
         assert torch.allclose(a, x.grad, rtol=1e-5, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# GEGLU expert (GLU in the feed-forward layer)
+# ---------------------------------------------------------------------------
+
+def _gelu(a):
+    return 0.5 * a * (1.0 + math.erf(a / math.sqrt(2.0)))
+
+
+def test_geglu_row_closed_form(oracle_lib):
+    # x = e_0 and one-hot weights make each pre-activation a chosen number, so
+    # H_i = GELU(g_i) * l_i by hand (GELU(1) = Phi(1) = 0.8413447460685429...)
+    d, f = 8, 4
+    g = [1.0, -1.0, 2.5, 0.0]
+    lin = [2.0, 3.0, -0.5, 7.0]
+    x = torch.zeros(d, dtype=torch.float32)
+    x[0] = 1.0
+    W1 = torch.zeros(2 * f, d, dtype=torch.float32)
+    for i in range(f):
+        W1[2 * i, 0] = g[i]
+        W1[2 * i + 1, 0] = lin[i]
+    W2 = torch.zeros(d, f, dtype=torch.float32)
+    for i in range(f):
+        W2[i, i] = 1.0  # out_i = H_i
+    out, H = oracle.expert_row(x, W1, W2, with_H=True, kind="geglu")
+    want = [_gelu(a) * b for a, b in zip(g, lin)]
+    assert _gelu(1.0) == pytest.approx(0.8413447460685429, rel=1e-15)
+    assert H.tolist() == [float(torch.tensor(v, dtype=torch.float32)) for v in want]
+    assert out[:f].tolist() == H.tolist() and float(out[f:].abs().sum()) == 0.0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_geglu_against_library_gelu(oracle_lib, dtype):
+    # an independent statement: torch's exact GELU on float64 products
+    d, f = 64, 96
+    x = synth.normal(8, 1, (d,), 1.0, dtype)
+    W1 = synth.normal(8, 3, (2 * f, d), 0.1, dtype)
+    W2 = synth.normal(8, 4, (d, f), 0.1, dtype)
+    out, H = oracle.expert_row(x, W1, W2, with_H=True, kind="geglu")
+    a = W1.double() @ x.double()
+    h_ref = torch.nn.functional.gelu(a[0::2], approximate="none") * a[1::2]
+    h_ref = h_ref.to(dtype)  # one rounding to the activation type
+    assert torch.equal(H, h_ref) or torch.allclose(H.double(), h_ref.double(), rtol=2 ** -7, atol=0)
+    o_ref = (W2.double() @ H.double()).to(dtype)
+    assert torch.allclose(out.double(), o_ref.double(), rtol=2 ** -7, atol=1e-30)
+
+
+def test_geglu_ffn_and_token_forward_agree(oracle_lib):
+    # the per-expert batch, the per-token path and the row function give the same rows
+    E, C, d, f = 3, 5, 64, 64
+    xe = synth.normal(9, 1, (E, C, d), 1.0, torch.bfloat16)
+    W1 = synth.normal(9, 3, (E, 2 * f, d), 0.05, torch.bfloat16)
+    W2 = synth.normal(9, 4, (E, d, f), 0.05, torch.bfloat16)
+    kept = torch.tensor([5, 0, 3], dtype=torch.int32)
+    ye = oracle.expert_ffn(xe, W1, W2, kept, kind="geglu")
+    for e in range(E):
+        for r in range(int(kept[e])):
+            row = oracle.expert_row(xe[e, r], W1[e], W2[e], kind="geglu")
+            assert torch.equal(ye[e, r], row)
+            y = oracle.token_forward(xe[e, r], W1, W2, torch.tensor([e], dtype=torch.int32),
+                                     torch.tensor([1.0]), torch.tensor([1], dtype=torch.uint8),
+                                     kind="geglu")
+            assert torch.equal(y, row)
