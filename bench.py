@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="switch_base", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--expert", default="relu", choices=["relu", "geglu"],
+                    help="expert network (the workloads are defined with the ReLU FFN)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -169,7 +171,7 @@ def oracle_step_fn(w, T_s):
     def step():
         oracle.layer_forward(inp["x"], inp["W1"], inp["W2"], E=ws.E, k=ws.k, C=C, Wr=inp["Wr"],
                              bias=inp["bias"], domain=inp["domain"], G=ws.num_groups, seed=ws.seed,
-                             nthreads=nth)
+                             nthreads=nth, kind=ws.expert)
     return step, nth
 
 
@@ -265,7 +267,9 @@ def stage_work(w, C, es, n_kept, tok_any):
     if fused_combine:
         disp += (T - tok_any) * d * es                    # dropped tokens' output rows zeroed
     st["dispatch"] = (disp, 0.0)
-    st["expert_ffn"] = (2 * E * d * f * es + 2 * n_kept * d * es, 4.0 * n_kept * d * f)
+    glu = w.expert == "geglu"  # W1 has 2f rows: 3 weight matrices' worth, 6 d f flops per row
+    st["expert_ffn"] = ((3 if glu else 2) * E * d * f * es + 2 * n_kept * d * es,
+                        (6.0 if glu else 4.0) * n_kept * d * f)
     st["combine"] = (0 if fused_combine else (n_kept + T) * d * es + 9 * T * k, 0.0)
     return st
 
@@ -294,7 +298,7 @@ def run_b200(args, w, world, rank, local):
     es = 2 if w.dtype == "bf16" else 4
     C = moe.capacity(w.T, w.E, w.capacity_factor)
     cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, C, dtype=w.torch_dtype, mode=w.mode,
-                          num_groups=w.num_groups, seed=w.seed)
+                          num_groups=w.num_groups, seed=w.seed, expert=w.expert)
     inp = synth.layer_inputs(w, x_seed_offset=rank)
     W1, W2 = inp["W1"].to(dev), inp["W2"].to(dev)
     Wr = None if inp["Wr"] is None else inp["Wr"].to(dev)
@@ -401,7 +405,7 @@ def run_b200(args, w, world, rank, local):
         roof = {"bound": "tensor", "achieved": ffn_flops / ffn_s / 1e12,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    tr = FFN_TRAFFIC.get(w.name)
+    tr = FFN_TRAFFIC.get(w.name) if w.expert == "relu" else None
     roof["traffic"] = tr[0] if tr else None
     roof["traffic_unit"] = "bytes per expert-FFN stage (ncu dram__bytes_read + write)"
     roof["traffic_source"] = tr[1] if tr else None
@@ -562,6 +566,7 @@ def run_b200(args, w, world, rank, local):
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E,
                    "k": w.k, "capacity_factor": w.capacity_factor, "capacity": C,
+                   "expert": w.expert,
                    "routing": w.mode, "tokens_per_rank_per_step": w.T,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"x rotated over {n_rot} batches ({n_rot * x_bytes / 2**20:.0f} MiB) and "
@@ -593,6 +598,8 @@ def run_b200(args, w, world, rank, local):
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
+    if args.expert != "relu":
+        w = w.scaled(expert=args.expert)
     world, rank, local = (1, 0, 0)
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -48,6 +48,8 @@ constexpr uint32_t kIdesc = dev::idesc_bf16_f32(kBM, kBN);
 
 struct FfnParams {
   int E, C, d, f, lag;
+  int n1;                  // GEMM-1 output columns: f (ReLU) or 2f (GEGLU: gate/linear pairs)
+  int glu;                 // 1: GEGLU expert
   const int32_t* kept_cnt;
   __nv_bfloat16* H;
   __nv_bfloat16* ye;
@@ -153,7 +155,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
   Sched sc;
   sc.E = E;
   sc.lag = p.lag;
-  sc.nb1 = (p.f + kBN - 1) / kBN;
+  sc.nb1 = (p.n1 + kBN - 1) / kBN;
   sc.nb2 = (p.d + kBN - 1) / kBN;
   sc.mblk = s_mblk;
   sc.prefix = s_prefix;
@@ -232,7 +234,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         const CUtensorMap* ta = x.kind == 1 ? &tmX : &tmH;
         const CUtensorMap* tb = x.kind == 1 ? &tmW1 : &tmW2;
         const int K = x.kind == 1 ? p.d : p.f;
-        const int b_rows = x.kind == 1 ? p.f : p.d;
+        const int b_rows = x.kind == 1 ? p.n1 : p.d;
         if (x.kind == 2) {
           // all GEMM-1 tiles of this expert must have stored H (4 warp arrivals per tile)
           const unsigned int need = static_cast<unsigned int>(4 * s_mblk[x.e] * sc.nb1);
@@ -333,26 +335,30 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       const int rows_valid = s_rows[x.e] - x.m * kBM;
       const bool row_ok = row_local < rows_valid;
       const int64_t grow = static_cast<int64_t>(x.e) * p.C + x.m * kBM + row_local;
-      const int N = x.kind == 1 ? p.f : p.d;
-      __nv_bfloat16* out = (x.kind == 1 ? p.H : p.ye) + grow * N;
+      const int N = x.kind == 1 ? p.n1 : p.d;       // this GEMM's output columns
+      const int ld = x.kind == 1 ? p.f : p.d;        // row stride of H / ye / y
+      __nv_bfloat16* out = (x.kind == 1 ? p.H : p.ye) + grow * ld;
       float scale = 1.f;
       if (x.kind == 2 && p.y && row_ok) {
         // top-1 combine (eq. 2 with one expert): y[t] = gate_t * E(x_t), into token order
         const int tok = __ldg(p.tok_of_row + grow);
         scale = __ldg(p.gate + tok);
-        out = p.y + static_cast<int64_t>(tok) * N;
+        out = p.y + static_cast<int64_t>(tok) * ld;
       }
       const int n0 = x.n * kBN;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * kAccStride);
       const bool relu = x.kind == 1;
+      const bool glu = x.kind == 1 && p.glu;
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t r[32];
         dev::tmem_ld_32x32b_x32(tbase + c * 32, r);
         dev::tmem_wait_ld();
         const int n = n0 + c * 32;
-        if (row_ok && n < N) {
+        if (glu) {
+          if (row_ok && n < N) dev::store_geglu16(r, out + n / 2);
+        } else if (row_ok && n < N) {
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -455,14 +461,16 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
     cudaError_t e = cudaMemsetAsync(sync, 0, ffn_sync_bytes(c), s);
     if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("cudaMemsetAsync: ") + cudaGetErrorString(e));
   }
+  const bool glu = c.expert == MOE_EXPERT_GEGLU;
+  const int64_t n1 = glu ? 2 * f : f;  // W1 rows per expert
   CUtensorMap tx, tw1, th, tw2;
   int32_t rc = make_tmap(&tx, xe, static_cast<uint64_t>(E * C), static_cast<uint64_t>(d), kBM);
-  if (rc == MOE_OK) rc = make_tmap(&tw1, W1, static_cast<uint64_t>(E * f), static_cast<uint64_t>(d), kBN);
+  if (rc == MOE_OK) rc = make_tmap(&tw1, W1, static_cast<uint64_t>(E * n1), static_cast<uint64_t>(d), kBN);
   if (rc == MOE_OK) rc = make_tmap(&th, H, static_cast<uint64_t>(E * C), static_cast<uint64_t>(f), kBM);
   if (rc == MOE_OK) rc = make_tmap(&tw2, W2, static_cast<uint64_t>(E * d), static_cast<uint64_t>(f), kBN);
   if (rc != MOE_OK) return rc;
   const int64_t mblk_max = (C + kBM - 1) / kBM;
-  const int64_t nb1 = (f + kBN - 1) / kBN, nb2 = (d + kBN - 1) / kBN;
+  const int64_t nb1 = (n1 + kBN - 1) / kBN, nb2 = (d + kBN - 1) / kBN;
   const int64_t g1_per_expert = mblk_max * nb1;
   const int sms = num_sms();
   // lag: GEMM-2 tiles of expert e come after ~2 waves of GEMM-1 tiles of later experts
@@ -473,6 +481,8 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
   p.C = c.capacity;
   p.d = c.d_model;
   p.f = c.d_ff;
+  p.n1 = static_cast<int>(n1);
+  p.glu = glu ? 1 : 0;
   p.lag = lag;
   p.kept_cnt = kept_cnt;
   p.H = static_cast<__nv_bfloat16*>(H);

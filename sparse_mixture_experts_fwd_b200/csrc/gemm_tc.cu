@@ -28,7 +28,9 @@ namespace {
 
 // EPI_TOPK: the router's epilogue computes the gate and top-k itself (Switch
 // notes sec. 2.1, eq. 1) from the token's logits in TMEM instead of storing them.
-enum EpiKind { EPI_RELU_BF16 = 0, EPI_BF16 = 1, EPI_F32_BIAS = 2, EPI_TOPK = 3 };
+// EPI_GLU_BF16: GEMM 1 of a GEGLU expert; accumulator columns 2i, 2i + 1 are
+// hidden unit i's gate and linear parts, out gets GELU(gate) * linear.
+enum EpiKind { EPI_RELU_BF16 = 0, EPI_BF16 = 1, EPI_F32_BIAS = 2, EPI_TOPK = 3, EPI_GLU_BF16 = 4 };
 
 constexpr int kBM = 128;          // rows per tile (MMA M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
@@ -375,7 +377,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           dev::tmem_ld_32x32b_x32(tbase + c * 32, r);
           dev::tmem_wait_ld();
           const int n = n0 + c * 32;
-          if (row_ok && n < p.N) {
+          if (EPI == EPI_GLU_BF16) {
+            if (row_ok && n < p.N) dev::store_geglu16(r, out + n / 2);
+          } else if (row_ok && n < p.N) {
             uint32_t packed[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -483,14 +487,18 @@ int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1,
   p.max_rows = c.capacity;
   p.status = status;
   p.bias = nullptr;
-  // GEMM 1: [E*C, d] x [E*f, d]^T -> H [E*C, f], ReLU
-  p.N = c.d_ff;
-  p.b_group_rows = c.d_ff;
+  // GEMM 1: [E*C, d] x [E*f, d]^T -> H [E*C, f], ReLU; GEGLU: W1 has 2f rows
+  // per expert and each pair of accumulator columns gives one unit of H
+  const bool glu = c.expert == MOE_EXPERT_GEGLU;
+  const int64_t n1 = glu ? 2 * f : f;
+  p.N = static_cast<int32_t>(n1);
+  p.b_group_rows = static_cast<int32_t>(n1);
   p.K = c.d_model;
   p.out = H;
   p.out_ld = f;
-  int32_t rc = launch_gemm<256, EPI_RELU_BF16>(xe, E * C, W1, E * f, p,
-                                               E * mblk_max * ((f + 255) / 256), s);
+  const int64_t t1 = E * mblk_max * ((n1 + 255) / 256);
+  int32_t rc = glu ? launch_gemm<256, EPI_GLU_BF16>(xe, E * C, W1, E * n1, p, t1, s)
+                   : launch_gemm<256, EPI_RELU_BF16>(xe, E * C, W1, E * n1, p, t1, s);
   if (rc != MOE_OK) return rc;
   // GEMM 2: [E*C, f] x [E*d, f]^T -> ye [E*C, d]
   p.N = c.d_model;

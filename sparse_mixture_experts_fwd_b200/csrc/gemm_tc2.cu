@@ -42,7 +42,8 @@ constexpr int kMaxGroups = 256;
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
 constexpr uint32_t kIdesc = dev::idesc_bf16_f32(kBM, kBN);
 
-enum Epi2 { EPI2_RELU_BF16 = 0, EPI2_BF16 = 1 };
+// EPI2_GLU_BF16: GEMM 1 of a GEGLU expert (column pairs -> GELU(gate) * linear)
+enum Epi2 { EPI2_RELU_BF16 = 0, EPI2_BF16 = 1, EPI2_GLU_BF16 = 2 };
 
 struct Gemm2Params {
   int32_t num_groups;
@@ -310,7 +311,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         dev::tmem_ld_32x32b_x32(tbase + c * 32, r);
         dev::tmem_wait_ld();
         const int n = n0 + c * 32;
-        if (row_ok && n < p.N) {
+        if (EPI == EPI2_GLU_BF16) {
+          if (row_ok && n < p.N) dev::store_geglu16(r, out + n / 2);
+        } else if (row_ok && n < p.N) {
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -429,13 +432,17 @@ int32_t launch_ffn_pairs(const moe_config& c, const void* xe, const void* W1, co
   p.group_rows = kept_cnt;
   p.max_rows = c.capacity;
   p.status = status;
-  p.N = c.d_ff;
-  p.b_group_rows = c.d_ff;
+  // GEGLU: W1 has 2f rows per expert, each accumulator column pair one unit of H
+  const bool glu = c.expert == MOE_EXPERT_GEGLU;
+  const int64_t n1 = glu ? 2 * f : f;
+  p.N = static_cast<int32_t>(n1);
+  p.b_group_rows = static_cast<int32_t>(n1);
   p.K = c.d_model;
   p.out = static_cast<__nv_bfloat16*>(H);
   p.out_ld = f;
-  int32_t rc = launch_pair<EPI2_RELU_BF16>(xe, E * C, W1, E * f, p,
-                                           E * mblk_max * ((f + kBN - 1) / kBN), s);
+  const int64_t t1 = E * mblk_max * ((n1 + kBN - 1) / kBN);
+  int32_t rc = glu ? launch_pair<EPI2_GLU_BF16>(xe, E * C, W1, E * n1, p, t1, s)
+                   : launch_pair<EPI2_RELU_BF16>(xe, E * C, W1, E * n1, p, t1, s);
   if (rc != MOE_OK) return rc;
   p.N = c.d_model;
   p.b_group_rows = c.d_model;

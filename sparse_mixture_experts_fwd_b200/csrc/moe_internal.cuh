@@ -291,5 +291,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+
+// GEGLU hidden unit from its gate and linear accumulators (GEMM-1 columns 2i
+// and 2i + 1): GELU(g) * l with GELU(a) = a * Phi(a) = a (1 + erf(a / sqrt 2)) / 2.
+MOE_DEV float geglu(float g, float l) {
+  return 0.5f * g * (1.0f + erff(g * 0.70710678118654752f)) * l;
+}
+// 32 GEMM-1 accumulator columns (16 gate / linear pairs) -> 16 bf16 hidden
+// units stored at dst (32 bytes, 16-byte aligned).
+MOE_DEV void store_geglu16(const uint32_t (&r)[32], __nv_bfloat16* dst) {
+  uint32_t packed[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float h0 = geglu(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+    const float h1 = geglu(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+    __nv_bfloat162 h = __floats2bfloat162_rn(h0, h1);
+    packed[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  d[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+}
+
 }  // namespace dev
 }  // namespace moe

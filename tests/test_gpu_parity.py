@@ -54,7 +54,8 @@ def case(moe, cuda_device, request):
 
 def make_cfg(moe, w, C, T=None):
     return moe.make_config(w.T if T is None else T, w.d_model, w.d_ff, w.E, w.k, C,
-                           dtype=w.torch_dtype, mode=w.mode, num_groups=w.num_groups, seed=w.seed)
+                           dtype=w.torch_dtype, mode=w.mode, num_groups=w.num_groups, seed=w.seed,
+                           expert=w.expert)
 
 
 def zero_status(dev):
@@ -244,6 +245,37 @@ def test_expert_ffn_ragged_tiles(moe, cuda_device, dtype, shape):
         assert bool(torch.isnan(H[e, n:].float()).all()) and bool(torch.isnan(ye[e, n:].float()).all())
 
 
+@pytest.mark.parametrize("shape", sorted(FFN_SHAPES))
+def test_expert_ffn_geglu(moe, cuda_device, shape):
+    """GEGLU experts (W1 [E, 2f, d] gate/linear rows) on every FFN kernel's tiles."""
+    dev = cuda_device
+    E, C, d, f, kept_list = FFN_SHAPES[shape]
+    kept = torch.tensor(kept_list, dtype=torch.int32)
+    dt = torch.bfloat16
+    xe = synth.normal(22, 1, (E, C, d), 1.0, dt)
+    W1 = synth.normal(22, 3, (E, 2 * f, d), 0.1, dt)
+    W2 = synth.normal(22, 4, (E, d, f), 0.05, dt)
+    cfg = moe.make_config(1, d, f, E, 1, C, dtype=dt, expert="geglu")
+    H = torch.full((E, C, f), float("nan"), dtype=dt, device=dev)
+    ye = torch.full((E, C, d), float("nan"), dtype=dt, device=dev)
+    st = zero_status(dev)
+    moe.expert_ffn(cfg, xe.to(dev), W1.to(dev), W2.to(dev), kept.to(dev), H=H, ye=ye, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ye_ref, H_ref = oracle.expert_ffn(xe, W1, W2, kept, with_H=True, nthreads=threads(),
+                                      kind="geglu")
+    H, ye = H.cpu(), ye.cpu()
+    for e in range(E):
+        n = int(kept[e])
+        assert_close(H[e, :n], H_ref[e, :n], what=f"H[{e}]")
+        assert_close(ye[e, :n], ye_ref[e, :n], what=f"ye[{e}]")
+        for a, b in ((H[e, :n], H_ref[e, :n]), (ye[e, :n], ye_ref[e, :n])):
+            if a.numel():
+                far = (a.double() - b.double()).abs() > 2.0 ** -7 * b.double().abs() + 1e-3
+                assert float(far.double().mean()) < 1e-3
+        assert bool(torch.isnan(H[e, n:].float()).all()) and bool(torch.isnan(ye[e, n:].float()).all())
+
+
 # ---------------------------------------------------------------------------
 # the whole layer at full size, sampled outputs
 # ---------------------------------------------------------------------------
@@ -352,6 +384,10 @@ SMALL = [
     ("tiny_fp32_top2", 400, 32, 48, 8, 2, 1.5, "topk", 1, 0.0),
     ("odd_experts_top2", 500, 64, 128, 40, 2, 1.0, "topk", 1, 0.0),
     ("seven_experts", 300, 128, 64, 7, 1, 1.0, "topk", 1, 0.0),
+    # GEGLU experts in each FFN kernel: fused (C = 62), two launches (C = 300), SM pairs (C = 550)
+    ("geglu_top1", 1000, 128, 256, 16, 1, 1.0, "topk", 1, 0.0),
+    ("geglu_top2_multi_block", 1200, 128, 128, 8, 2, 2.0, "topk", 1, 0.0),
+    ("geglu_rre_pairs", 4400, 64, 128, 8, 1, 1.0, "rre", 2, 0.0),
 ]
 
 
@@ -361,12 +397,14 @@ def test_layer_small_cases(moe, cuda_device, case):
     dev = cuda_device
     dtype = "f32" if "fp32" in name else "bf16"
     w = synth.Workload(name, T=T, d_model=d, d_ff=f, E=E, k=k, capacity_factor=cf_, dtype=dtype,
-                       mode=mode, num_groups=G, hot_experts=1 if hot else 0, hot_bias=hot, seed=3)
+                       mode=mode, num_groups=G, hot_experts=1 if hot else 0, hot_bias=hot, seed=3,
+                       expert="geglu" if "geglu" in name else "relu",
+                       expert_std=0.1 if "geglu" in name else 0.02)
     inp = synth.layer_inputs(w)
     C = oracle.capacity(T, E, cf_)
     r = oracle.layer_forward(inp["x"], inp["W1"], inp["W2"], E=E, k=k, C=C, Wr=inp["Wr"],
                              bias=inp["bias"], domain=inp["domain"], G=G, seed=w.seed, with_H=True,
-                             nthreads=threads())
+                             nthreads=threads(), kind=w.expert)
     cfg = make_cfg(moe, w, C)
     ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
     st = zero_status(dev)
