@@ -244,8 +244,17 @@ __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArg
     if (s_ok < 0) return;  // bounded wait expired: outputs are invalid, status says so
     const int pstar = s_pstar;
     for (int x = tid; x < E; x += kAssignBlock) {
+      // the aggregates after p* are independent loads: 8 in flight per round
       int acc = __ldcg(p.incl + static_cast<int64_t>(pstar) * E + x);
-      for (int q = pstar + 1; q < b; ++q) acc += __ldcg(p.aggr + static_cast<int64_t>(q) * E + x);
+      int part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int q = pstar + 1;
+      for (; q + 8 <= b; q += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part[u] += __ldcg(p.aggr + static_cast<int64_t>(q + u) * E + x);
+      }
+      for (; q < b; ++q) part[0] += __ldcg(p.aggr + static_cast<int64_t>(q) * E + x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc += part[u];
       s_excl[x] = acc;
       p.incl[static_cast<int64_t>(b) * E + x] = acc + p.aggr[static_cast<int64_t>(b) * E + x];
     }
@@ -290,11 +299,10 @@ __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArg
       for (int w = 0; w < 32; ++w) tot += s_drop[w];
       p.n_dropped[0] = tot;
     }
-    const int64_t rows = static_cast<int64_t>(E) * p.C;
-    for (int64_t i = tid; i < rows; i += kAssignBlock) {
-      const int ex = static_cast<int>(i / p.C);
-      if (static_cast<int>(i - static_cast<int64_t>(ex) * p.C) >= s_cnt[ex]) p.tok_of_row[i] = -1;
-    }
+    // free rows of the map: a warp per expert, lanes over its rows past the kept count
+    for (int ex = warp; ex < E; ex += kAssignBlock / 32)
+      for (int r = s_cnt[ex] + lane; r < p.C; r += 32)
+        p.tok_of_row[static_cast<int64_t>(ex) * p.C + r] = -1;
   }
 }
 
