@@ -7,14 +7,16 @@
 // with p(x) the softmax of eq. (1) over all E experts and the argmax taken on
 // the fp32 logits, ties to the lower index (the top-1 choice).
 //
-// Pass 1 (HBM-bound: reads the logits once): a warp per token, two tokens in
-// flight per warp, E <= 256 logits held 8 per lane (coalesced); max/argmax
-// and the softmax sum by shuffles; each lane accumulates p for its experts
-// in double across the warp's tokens, the argmax is counted in shared
-// memory, H(p) = ln(s) - sum_e p_e (h_e - m) per token.  Each block (at most
-// four per SM) writes its partial P[E], counts[E] and entropy sum.  Pass 2: a
-// block per expert adds that expert's partials (strided, then a fixed tree:
-// deterministic).  Pass 3 (one block): sum_e f_e P_e and the entropy.
+// Pass 1 (HBM-bound: reads the logits once): a warp per token, the logits of
+// four tokens per warp loaded before any is reduced, E <= 256 logits held 8
+// per lane (coalesced); max/argmax and the softmax sum by shuffles; each lane
+// accumulates p for its experts in double across the warp's tokens, the
+// argmax is counted in shared memory, H(p) = ln(s) - sum_e p_e (h_e - m) per
+// token.  Each block (three per SM, one wave) writes its partial P[E], counts[E]
+// and entropy sum.  Pass 2: a block per expert adds that expert's partials
+// (strided, then a fixed tree: deterministic); the last block to finish
+// (a counter that pass 1 zeroes) forms sum_e f_e P_e and the entropy, in a
+// fixed order.
 #include <climits>
 #include <cmath>
 
@@ -25,10 +27,12 @@ namespace {
 
 constexpr int kAuxThreads = 256;  // 8 warps
 constexpr int kAuxWarps = kAuxThreads / 32;
+constexpr int kAuxInFlight = 4;  // tokens per warp whose logits are loaded together
+constexpr int kAuxBlocksPerSm = 3;  // 3 x 256 threads x <= 85 registers fill the register file
 
-__global__ void __launch_bounds__(kAuxThreads) aux_partial_kernel(
+__global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kernel(
     int64_t T, int E, const float* __restrict__ logits, double* __restrict__ part_P,
-    int32_t* __restrict__ part_cnt, double* __restrict__ part_H) {
+    int32_t* __restrict__ part_cnt, double* __restrict__ part_H, unsigned* __restrict__ done) {
   __shared__ double s_P[kAuxWarps][256];
   __shared__ int s_cnt[256];
   __shared__ double s_H[kAuxWarps];
@@ -36,19 +40,22 @@ __global__ void __launch_bounds__(kAuxThreads) aux_partial_kernel(
   dev::pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < 256; e += kAuxThreads) s_cnt[e] = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // pass 2's finishing counter
   __syncthreads();
   double accP[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   double accH = 0.0;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kAuxWarps;
-  // one token's softmax statistics; the caller keeps two in flight
-  auto token = [&](int64_t t) {
+  // one token's logits, lane + 32 q for q < 8 (-inf past E)
+  auto load = [&](int64_t t, float (&v)[8]) {
     const float* h = logits + t * E;
-    float v[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int e = lane + 32 * q;
       v[q] = e < E ? __ldg(h + e) : -INFINITY;
     }
+  };
+  // one token's softmax statistics
+  auto token = [&](const float (&v)[8]) {
     // argmax with the lower index on ties: each lane scans its experts in
     // ascending order with a strict compare, then a shuffle reduction
     float bv = -INFINITY;
@@ -88,12 +95,20 @@ __global__ void __launch_bounds__(kAuxThreads) aux_partial_kernel(
       accH += static_cast<double>(logf(s)) - static_cast<double>(w * inv);
     }
   };
+  // the warp's tokens t, t + nwarps, ... in that order, kAuxInFlight at a time
   int64_t t = static_cast<int64_t>(blockIdx.x) * kAuxWarps + warp;
-  for (; t + nwarps < T; t += 2 * nwarps) {
-    token(t);
-    token(t + nwarps);
+  for (; t + (kAuxInFlight - 1) * nwarps < T; t += kAuxInFlight * nwarps) {
+    float v[kAuxInFlight][8];
+#pragma unroll
+    for (int u = 0; u < kAuxInFlight; ++u) load(t + u * nwarps, v[u]);
+#pragma unroll
+    for (int u = 0; u < kAuxInFlight; ++u) token(v[u]);
   }
-  if (t < T) token(t);
+  for (; t < T; t += nwarps) {
+    float v[8];
+    load(t, v);
+    token(v);
+  }
 #pragma unroll
   for (int q = 0; q < 8; ++q) s_P[warp][lane + 32 * q] = accP[q];
   if (lane == 0) s_H[warp] = accH;
@@ -115,15 +130,21 @@ __global__ void __launch_bounds__(kAuxThreads) aux_partial_kernel(
 
 // Pass 2: block e adds expert e's partials over the pass-1 blocks (thread i
 // takes blocks i, i + 256, ..., then a fixed tree), f_e = count / T,
-// P_e = sum / T; fe_Pe[e] = f_e * P_e for pass 3.
-__global__ void __launch_bounds__(256) aux_reduce_kernel(int64_t T, int E, int nblk,
+// P_e = sum / T, fe_Pe[e] = f_e * P_e.  The block that finishes last (by the
+// counter pass 1 zeroed) forms loss = alpha * E * sum_e f_e P_e and
+// entropy = sum of the pass-1 entropy sums / T, both by fixed trees.
+__global__ void __launch_bounds__(256, 1) aux_reduce_kernel(int64_t T, int E, int nblk, double alpha,
                                                          const double* __restrict__ part_P,
                                                          const int32_t* __restrict__ part_cnt,
-                                                         double* __restrict__ fe_Pe,
+                                                         const double* __restrict__ part_H,
+                                                         double* fe_Pe, unsigned* done,
                                                          double* __restrict__ f_out,
-                                                         double* __restrict__ P_out) {
+                                                         double* __restrict__ P_out,
+                                                         double* __restrict__ out) {
   __shared__ double s_p[256];
   __shared__ long long s_c[256];
+  __shared__ double s_h[256];
+  __shared__ bool s_last;
   dev::pdl_trigger();
   dev::pdl_wait();
   const int e = blockIdx.x;
@@ -150,50 +171,46 @@ __global__ void __launch_bounds__(256) aux_reduce_kernel(int64_t T, int E, int n
     if (f_out) f_out[e] = fe;
     if (P_out) P_out[e] = Pe;
     fe_Pe[e] = fe * Pe;
+    __threadfence();  // fe_Pe[e] visible before this block counts as done
+    s_last = atomicAdd(done, 1u) == static_cast<unsigned>(E - 1);
   }
-}
-
-// Pass 3: loss = alpha * E * sum_e f_e P_e, entropy = sum of the blocks' sums / T.
-__global__ void __launch_bounds__(256) aux_final_kernel(int64_t T, int E, int nblk, double alpha,
-                                                        const double* __restrict__ fe_Pe,
-                                                        const double* __restrict__ part_H,
-                                                        double* __restrict__ out) {
-  __shared__ double s_d[256], s_h[256];
-  dev::pdl_trigger();
-  dev::pdl_wait();
-  double d = 0.0, h = 0.0;
-  for (int e = threadIdx.x; e < E; e += 256) d += fe_Pe[e];
-  for (int b = threadIdx.x; b < nblk; b += 256) h += part_H[b];
-  s_d[threadIdx.x] = d;
-  s_h[threadIdx.x] = h;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  double d = 0.0, hs = 0.0;
+  for (int q = threadIdx.x; q < E; q += 256) d += __ldcg(fe_Pe + q);
+  for (int b = threadIdx.x; b < nblk; b += 256) hs += part_H[b];
+  s_p[threadIdx.x] = d;  // s_p[0] was read before the last barrier
+  s_h[threadIdx.x] = hs;
   __syncthreads();
   for (int k = 128; k > 0; k >>= 1) {
     if (threadIdx.x < k) {
-      s_d[threadIdx.x] += s_d[threadIdx.x + k];
+      s_p[threadIdx.x] += s_p[threadIdx.x + k];
       s_h[threadIdx.x] += s_h[threadIdx.x + k];
     }
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    out[0] = alpha * static_cast<double>(E) * s_d[0];
+    out[0] = alpha * static_cast<double>(E) * s_p[0];
     out[1] = T > 0 ? s_h[0] / static_cast<double>(T) : 0.0;
   }
 }
 
 int aux_blocks(const moe_config& c) {
   const int64_t want = (c.T + kAuxWarps * 4 - 1) / (kAuxWarps * 4);  // >= 4 tokens per warp
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 4;  // 4 blocks of 256 per SM fit
+  const int64_t cap = static_cast<int64_t>(num_sms()) * kAuxBlocksPerSm;  // one wave
   return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
 }  // namespace
 
 // per block: P [E] double, counts [E] int32; then the entropy sums [nblk]
-// double; then f_e P_e [E] double
+// double; then f_e P_e [E] double; then pass 2's finishing counter
 size_t aux_workspace_bytes(const moe_config& c) {
   const size_t nblk = static_cast<size_t>(aux_blocks(c));
   return align256(nblk * c.E * sizeof(double)) + align256(nblk * c.E * sizeof(int32_t)) +
-         align256(nblk * sizeof(double)) + align256(static_cast<size_t>(c.E) * sizeof(double));
+         align256(nblk * sizeof(double)) + align256(static_cast<size_t>(c.E) * sizeof(double)) +
+         align256(sizeof(unsigned));
 }
 
 int32_t launch_aux_loss(const moe_config& c, const float* logits, double alpha, double* out,
@@ -207,17 +224,15 @@ int32_t launch_aux_loss(const moe_config& c, const float* logits, double alpha, 
   int32_t* part_cnt = reinterpret_cast<int32_t*>(ws + bP);
   double* part_H = reinterpret_cast<double*>(ws + bP + bC);
   double* fe_Pe = reinterpret_cast<double*>(ws + bP + bC + bH);
+  unsigned* done = reinterpret_cast<unsigned*>(ws + bP + bC + bH + align256(static_cast<size_t>(c.E) * 8));
   launch_pdl(aux_partial_kernel, dim3(static_cast<unsigned>(nblk)), dim3(kAuxThreads), 0, s, c.T,
-             c.E, logits, part_P, part_cnt, part_H);
+             c.E, logits, part_P, part_cnt, part_H, done);
   int32_t rc = check_launch("aux_partial_kernel");
   if (rc != MOE_OK) return rc;
   launch_pdl(aux_reduce_kernel, dim3(static_cast<unsigned>(c.E)), dim3(256), 0, s, c.T, c.E, nblk,
-             static_cast<const double*>(part_P), static_cast<const int32_t*>(part_cnt), fe_Pe, f, P);
-  rc = check_launch("aux_reduce_kernel");
-  if (rc != MOE_OK) return rc;
-  launch_pdl(aux_final_kernel, dim3(1), dim3(256), 0, s, c.T, c.E, nblk, alpha,
-             static_cast<const double*>(fe_Pe), static_cast<const double*>(part_H), out);
-  return check_launch("aux_final_kernel");
+             alpha, static_cast<const double*>(part_P), static_cast<const int32_t*>(part_cnt),
+             static_cast<const double*>(part_H), fe_Pe, done, f, P, out);
+  return check_launch("aux_reduce_kernel");
 }
 
 }  // namespace moe

@@ -489,8 +489,8 @@ def test_layer_zero_tokens(moe, cuda_device):
 # Switch load-balancing loss (eqs. 4-6) and routing entropy
 # ---------------------------------------------------------------------------
 
-def _check_aux(moe, cfg, logits, alpha=1e-2):
-    out, f, P = moe.aux_loss(cfg, logits.to("cuda"), alpha)
+def _check_aux(moe, cfg, logits, alpha=1e-2, workspace=None):
+    out, f, P = moe.aux_loss(cfg, logits.to("cuda"), alpha, workspace=workspace)
     torch.cuda.synchronize()
     loss, ent, f_ref, P_ref = oracle.aux_loss(logits.cpu().contiguous(), alpha)
     # the same fp32 logits and tie rule on both sides: f (token counts / T) is exact
@@ -507,12 +507,23 @@ def test_aux_loss_full(moe, cuda_device, case):
     _check_aux(moe, case.cfg, case.ref["logits"])
 
 
-@pytest.mark.parametrize("T,E", [(1, 1), (1, 8), (1000, 40), (4097, 256), (300, 7)])
+@pytest.mark.parametrize("T,E", [(1, 1), (1, 8), (1000, 40), (4097, 256), (300, 7), (40000, 64)])
 def test_aux_loss_shapes(moe, cuda_device, T, E):
     cfg = moe.make_config(T, 64, 64, E, 1, 1, dtype=torch.float32)
     _check_aux(moe, cfg, synth.normal(3, 2, (T, E), 2.0, torch.float32))
     # equal logits: every argmax is expert 0 and the loss is exactly alpha
     _check_aux(moe, cfg, torch.zeros(T, E))
+
+
+def test_aux_loss_reused_workspace(moe, cuda_device):
+    """One workspace, filled with 0xff bytes, for back-to-back calls on
+    different logits: the partials and the finishing counter are set up by
+    each call, so every call matches the oracle."""
+    T, E = 9000, 96
+    cfg = moe.make_config(T, 64, 64, E, 1, 1, dtype=torch.float32)
+    ws = torch.full((max(256, moe.aux_workspace_size(cfg)),), 255, dtype=torch.uint8, device="cuda")
+    for seed in (5, 6, 7):
+        _check_aux(moe, cfg, synth.normal(seed, 2, (T, E), 1.5, torch.float32), workspace=ws)
 
 
 def test_aux_loss_zero_tokens(moe, cuda_device):
