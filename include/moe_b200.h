@@ -66,7 +66,9 @@ enum moe_route_mode { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RRE = 1 };
 enum moe_expert { MOE_EXPERT_RELU = 0, MOE_EXPERT_GEGLU = 1 };
 enum moe_status_bits {
   MOE_STATUS_TIMEOUT = 1,   /* a pipeline wait gave up after 1 s; outputs invalid     */
-  MOE_STATUS_BAD_DOMAIN = 2 /* an RRE domain id was outside 0..G-1 (routed as 0)       */
+  MOE_STATUS_BAD_DOMAIN = 2, /* an RRE domain id was outside 0..G-1 (routed as 0)      */
+  MOE_STATUS_BAD_COUNTS = 4  /* expert parallel: a row fell outside its expert's block
+                                (counts that do not match the assignment); skipped     */
 };
 
 /* One MoE layer.  56 bytes, no padding. */
@@ -288,6 +290,66 @@ int32_t sparseclip_norm_noalloc(const float* const* dense, const int64_t* dense_
                                 int32_t n_dense, const float* const* sparse,
                                 const int64_t* sparse_len, int32_t n_sparse, int32_t num_experts,
                                 double* out, moe_stream_t stream);
+
+/* ---- expert parallelism over the GPUs of one node ---------------------- */
+
+/* The sparse layer's distinct expert weights placed on different devices
+ * (Switch notes sec. 2, opening paragraph: the parameter count grows with the
+ * device count while each device's memory and compute stay bounded).
+ * `world` ranks (1..8), El = E / world experts each: rank r holds experts
+ * r*El .. (r+1)*El - 1 (W1, W2 shards [El, ...]).  Every rank routes and
+ * assigns its own batch of cfg->T tokens exactly as moe_topk_assign does,
+ * with capacity C = cfg->capacity per batch, so each rank's output equals the
+ * single-device layer (moe_layer_forward) on that rank's batch.
+ *
+ * cnt_all [world, E] int32 (device): row q = the kept_cnt of rank q, exchanged
+ * by the caller (an all-gather) before the dispatch.
+ * Receive buffers: rank r's xe_r and ye_r are [El, world*C, d] in cfg->dtype.
+ * The kept rows for its local expert el from rank q sit at rows
+ * off_q(e) .. off_q(e) + cnt_all[q, e] - 1 of block el (e = r*El + el),
+ * off_q(e) = sum over q' < q of cnt_all[q', e]: rank order, then slot order.
+ *
+ * One layer step on rank r:
+ *   1. moe_router + moe_topk_assign on the rank's batch (global E);
+ *   2. all-gather of kept_cnt into cnt_all;
+ *   3. moe_ep_dispatch (stores rows into the home ranks' xe);
+ *   4. a barrier across ranks (every rank's dispatch complete);
+ *   5. moe_expert_ffn on xe_r with the config moe_ep_ffn_config gives and
+ *      kept counts local_cnt, writing ye_r;
+ *   6. a barrier across ranks (every rank's FFN complete);
+ *   7. moe_ep_combine (loads rows from the home ranks' ye).
+ * The library's kernels never wait on another rank: the caller's collectives
+ * in steps 2, 4 and 6 order the ranks. */
+
+/* The expert-FFN config of one rank: cfg with E = El, capacity = world*C
+ * (k, mode and num_groups set to 1, TOPK and 1: routing does not enter the
+ * FFN).  Host only.  MOE_ERR_INVALID_ARGUMENT if world is outside 1..8 or does
+ * not divide E; MOE_ERR_UNSUPPORTED if world*C exceeds 2^31-1. */
+int32_t moe_ep_ffn_config(const moe_config* cfg, int32_t world, moe_config* out);
+
+/* Step 3.  For each kept choice (t, j) of this rank, with e = expert_idx[t, j],
+ * h = e / El:  xe_h[e - h*El, off_rank(e) + slot[t, j], :] = x[t, :].
+ * xe_peers: host array of `world` device pointers, entry q = rank q's xe as
+ * mapped into this process (CUDA IPC or peer access; entry `rank` = this
+ * rank's own), each 16-byte aligned.  local_cnt [El] int32 (device,
+ * nullable): receives sum over q of cnt_all[q, rank*El + el], the kept counts
+ * for step 5.  A row whose index would fall outside 0..world*C-1 is skipped
+ * and sets MOE_STATUS_BAD_COUNTS.  x [T, d] in cfg->dtype. */
+int32_t moe_ep_dispatch(const moe_config* cfg, int32_t rank, int32_t world, const void* x,
+                        const int32_t* expert_idx, const int32_t* slot, const uint8_t* kept,
+                        const int32_t* cnt_all, void* const* xe_peers, int32_t* local_cnt,
+                        int32_t* status, moe_stream_t stream);
+
+/* Step 7, the combine of eq. 2 (Switch notes sec. 2.1) over the home ranks'
+ * outputs:  y[t, :] = sum over kept j of gate[t, j] *
+ * ye_h[e - h*El, off_rank(e) + slot[t, j], :], fp32 accumulation in choice
+ * order, one rounding; 0 for a token with no kept choice.  ye_peers: host
+ * array of `world` device pointers as for moe_ep_dispatch.  y [T, d] in
+ * cfg->dtype.  Out-of-block rows: skipped, MOE_STATUS_BAD_COUNTS. */
+int32_t moe_ep_combine(const moe_config* cfg, int32_t rank, int32_t world,
+                       const void* const* ye_peers, const int32_t* expert_idx, const float* gate,
+                       const int32_t* slot, const uint8_t* kept, const int32_t* cnt_all, void* y,
+                       int32_t* status, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

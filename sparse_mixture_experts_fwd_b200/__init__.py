@@ -23,7 +23,7 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARGUMENT", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ER
           -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 ROUTE_TOPK, ROUTE_RRE = 0, 1
-STATUS_TIMEOUT, STATUS_BAD_DOMAIN = 1, 2
+STATUS_TIMEOUT, STATUS_BAD_DOMAIN, STATUS_BAD_COUNTS = 1, 2, 4
 
 # every entry point the header declares, with its ctypes signature
 _i32, _i64, _u64, _sz, _vp, _dbl = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64,
@@ -46,6 +46,7 @@ class WorkspaceMap(ctypes.Structure):
 
 
 _PCFG = ctypes.POINTER(MoEConfig)
+_PVP = ctypes.POINTER(ctypes.c_void_p)
 SIGNATURES = {
     "moe_abi_version": ([], _i32),
     "moe_config_size": ([], _sz),
@@ -72,6 +73,9 @@ SIGNATURES = {
     "sparseclip_norm": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "sparseclip_norm_noalloc": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
     "sparseclip_clip": ([_vp, _vp, _i32, _vp, _vp, _i32, _i32, _dbl, _vp, _vp, _sz, _vp], _i32),
+    "moe_ep_ffn_config": ([_PCFG, _i32, _PCFG], _i32),
+    "moe_ep_dispatch": ([_PCFG, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _PVP, _vp, _vp, _vp], _i32),
+    "moe_ep_combine": ([_PCFG, _i32, _i32, _PVP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
 }
 
 
@@ -258,6 +262,63 @@ def combine(cfg, ye, expert_idx, gate, slot, kept, y=None, stream=None):
     _check(lib.moe_combine(ctypes.byref(cfg), _ptr(ye, "ye"), _ptr(expert_idx, "expert_idx"),
                            _ptr(gate, "gate"), _ptr(slot, "slot"), _ptr(kept, "kept"),
                            _ptr(y, "y"), _stream(stream)), "moe_combine")
+    return y
+
+
+def ep_ffn_config(cfg: MoEConfig, world: int) -> MoEConfig:
+    """The expert-FFN config of one of ``world`` expert-parallel ranks:
+    E / world experts, capacity world * C."""
+    out = MoEConfig()
+    _check(lib.moe_ep_ffn_config(ctypes.byref(cfg), int(world), ctypes.byref(out)),
+           "moe_ep_ffn_config")
+    return out
+
+
+def _peer_table(peers, world, name):
+    """Host array of ``world`` device addresses from tensors or ints (mapped peer pointers)."""
+    if peers is None:
+        return None
+    if len(peers) != world:
+        raise ValueError(f"{name} needs {world} entries, got {len(peers)}")
+    addr = []
+    for q, p in enumerate(peers):
+        if isinstance(p, torch.Tensor):
+            addr.append(_ptr(p, f"{name}[{q}]"))
+        else:
+            addr.append(int(p))
+    return (ctypes.c_void_p * world)(*addr)
+
+
+def ep_dispatch(cfg, rank, world, x, expert_idx, slot, kept, cnt_all, xe_peers, local_cnt=None,
+                status=None, stream=None):
+    """Expert-parallel dispatch: this rank's kept rows into their home ranks'
+    receive buffers ``xe_peers`` (tensors or mapped device addresses, rank
+    order).  Returns ``local_cnt`` [E / world], the rows each local expert
+    receives from all ranks."""
+    if local_cnt is None:
+        local_cnt = torch.empty(cfg.E // world, dtype=torch.int32, device=cnt_all.device)
+    _check(lib.moe_ep_dispatch(ctypes.byref(cfg), int(rank), int(world), _ptr(x, "x"),
+                               _ptr(expert_idx, "expert_idx"), _ptr(slot, "slot"),
+                               _ptr(kept, "kept"), _ptr(cnt_all, "cnt_all"),
+                               _peer_table(xe_peers, world, "xe_peers"),
+                               _ptr(local_cnt, "local_cnt"), _ptr(status, "status"),
+                               _stream(stream)), "moe_ep_dispatch")
+    return local_cnt
+
+
+def ep_combine(cfg, rank, world, ye_peers, expert_idx, gate, slot, kept, cnt_all, y=None,
+               status=None, stream=None):
+    """Expert-parallel combine: y [T, d] from the home ranks' expert outputs
+    ``ye_peers`` (tensors or mapped device addresses, rank order)."""
+    if y is None:
+        dt = torch.bfloat16 if cfg.dtype == DTYPE_BF16 else torch.float32
+        y = torch.empty(cfg.T, cfg.d_model, dtype=dt, device=cnt_all.device)
+    _check(lib.moe_ep_combine(ctypes.byref(cfg), int(rank), int(world),
+                              _peer_table(ye_peers, world, "ye_peers"),
+                              _ptr(expert_idx, "expert_idx"), _ptr(gate, "gate"),
+                              _ptr(slot, "slot"), _ptr(kept, "kept"), _ptr(cnt_all, "cnt_all"),
+                              _ptr(y, "y"), _ptr(status, "status"), _stream(stream)),
+           "moe_ep_combine")
     return y
 
 

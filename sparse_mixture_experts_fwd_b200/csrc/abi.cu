@@ -406,4 +406,82 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
   return mark(5);
 }
 
+namespace {
+
+int32_t check_ep(const moe_config* cfg, int32_t rank, int32_t world) {
+  MOE_TRY(check_cfg(cfg));
+  if (world < 1 || world > kMaxEpRanks)
+    return fail(MOE_ERR_INVALID_ARGUMENT, "world must be 1.." + std::to_string(kMaxEpRanks));
+  if (rank < 0 || rank >= world) return fail(MOE_ERR_INVALID_ARGUMENT, "rank outside 0..world-1");
+  if (cfg->E % world != 0) return fail(MOE_ERR_INVALID_ARGUMENT, "world does not divide E");
+  if (int64_t(world) * cfg->capacity > kI32Max)
+    return fail(MOE_ERR_UNSUPPORTED, "world * capacity exceeds 2^31-1 rows");
+  return MOE_OK;
+}
+
+int32_t check_peers(const void* const* peers, int32_t world, const char* name) {
+  if (!peers) return fail(MOE_ERR_INVALID_ARGUMENT, std::string(name) + " is null");
+  for (int q = 0; q < world; ++q)
+    MOE_TRY(need_ptr(peers[q], (std::string(name) + "[" + std::to_string(q) + "]").c_str()));
+  return MOE_OK;
+}
+
+}  // namespace
+
+int32_t moe_ep_ffn_config(const moe_config* cfg, int32_t world, moe_config* out) {
+  set_last_error("");
+  MOE_TRY(check_ep(cfg, 0, world));
+  if (!out) return fail(MOE_ERR_INVALID_ARGUMENT, "out is null");
+  moe_config c = *cfg;
+  c.E = cfg->E / world;
+  c.capacity = world * cfg->capacity;
+  c.k = 1;
+  c.mode = MOE_ROUTE_TOPK;
+  c.num_groups = 1;
+  MOE_TRY(check_cfg(&c));
+  *out = c;
+  return MOE_OK;
+}
+
+int32_t moe_ep_dispatch(const moe_config* cfg, int32_t rank, int32_t world, const void* x,
+                        const int32_t* expert_idx, const int32_t* slot, const uint8_t* kept,
+                        const int32_t* cnt_all, void* const* xe_peers, int32_t* local_cnt,
+                        int32_t* status, moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_ep(cfg, rank, world));
+  MOE_TRY(need_ptr4(cnt_all, "cnt_all"));
+  if (local_cnt) MOE_TRY(need_ptr4(local_cnt, "local_cnt"));
+  if (cfg->T > 0 && cfg->capacity > 0) {
+    MOE_TRY(need_ptr(x, "x"));
+    MOE_TRY(need_ptr4(expert_idx, "expert_idx"));
+    MOE_TRY(need_ptr4(slot, "slot"));
+    if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
+    MOE_TRY(check_peers(xe_peers, world, "xe_peers"));
+  } else if (!local_cnt) {
+    return MOE_OK;  // nothing to send and nothing to count
+  }
+  moe_config c = *cfg;
+  if (c.capacity == 0) c.T = 0;  // no choice is kept
+  return launch_ep_dispatch(c, rank, world, x, expert_idx, slot, kept, cnt_all, xe_peers,
+                            local_cnt, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_ep_combine(const moe_config* cfg, int32_t rank, int32_t world,
+                       const void* const* ye_peers, const int32_t* expert_idx, const float* gate,
+                       const int32_t* slot, const uint8_t* kept, const int32_t* cnt_all, void* y,
+                       int32_t* status, moe_stream_t stream) {
+  set_last_error("");
+  MOE_TRY(check_ep(cfg, rank, world));
+  if (cfg->T == 0) return MOE_OK;
+  MOE_TRY(need_ptr4(expert_idx, "expert_idx"));
+  MOE_TRY(need_ptr4(gate, "gate"));
+  MOE_TRY(need_ptr4(slot, "slot"));
+  if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
+  MOE_TRY(need_ptr4(cnt_all, "cnt_all"));
+  MOE_TRY(need_ptr(y, "y"));
+  if (cfg->capacity > 0) MOE_TRY(check_peers(ye_peers, world, "ye_peers"));
+  return launch_ep_combine(*cfg, rank, world, ye_peers, expert_idx, gate, slot, kept, cnt_all, y,
+                           status, reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

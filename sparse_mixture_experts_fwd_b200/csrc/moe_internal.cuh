@@ -98,6 +98,17 @@ int32_t launch_aux_loss(const moe_config& c, const float* logits, double alpha, 
 int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* expert_idx,
                        const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
                        cudaStream_t s);
+// expert parallelism over the ranks of one node: the receive buffers of all
+// ranks as mapped into this process, rank order
+constexpr int kMaxEpRanks = 8;
+int32_t launch_ep_dispatch(const moe_config& c, int rank, int world, const void* x,
+                           const int32_t* expert_idx, const int32_t* slot, const uint8_t* kept,
+                           const int32_t* cnt_all, void* const* xe_peers, int32_t* local_cnt,
+                           int32_t* status, cudaStream_t s);
+int32_t launch_ep_combine(const moe_config& c, int rank, int world, const void* const* ye_peers,
+                          const int32_t* expert_idx, const float* gate, const int32_t* slot,
+                          const uint8_t* kept, const int32_t* cnt_all, void* y, int32_t* status,
+                          cudaStream_t s);
 
 }  // namespace moe
 

@@ -9,6 +9,19 @@
 // gathers the k expert output rows with 16-byte loads, accumulates
 // gate * row in fp32 (choice order j = 0, 1) and writes the token's row once,
 // rounded to the activation type; a token with no kept choice gets zeros.
+//
+// Expert-parallel forms (Switch notes sec. 2, opening: the sparse layer's
+// distinct expert weights live on different devices, so the parameter count
+// grows with the device count): `world` ranks, rank r holds experts
+// r*El .. (r+1)*El - 1 and routes its own batch.  Expert e's rows on its home
+// rank h = e / El form one [world*C, d] block of the receive buffer
+// [El, world*C, d]; the rows from rank q start at off_q(e) = sum over q' < q
+// of q''s kept count of e, in q's slot (token) order.  ep_dispatch_kernel
+// stores each kept row straight into the home rank's buffer through its peer
+// mapping (NVLink stores; a plain store when h is this rank), and
+// ep_combine_kernel loads each token's expert outputs back the same way.
+// Neither waits on another rank: the caller orders dispatch -> expert FFN ->
+// combine across ranks (a collective between the steps).
 #include <algorithm>
 
 #include "moe_internal.cuh"
@@ -151,6 +164,147 @@ unsigned grid_for_tokens(int64_t T) {
   return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(num_sms()) * 16)));
 }
 
+// peer buffers of the ranks of one node, by rank
+struct PeerRows {
+  uint4* p[kMaxEpRanks];
+};
+struct PeerRowsConst {
+  const uint4* p[kMaxEpRanks];
+};
+
+// entry h of a kernel-parameter table, by selects (a dynamic index would copy
+// the table to local memory)
+template <class P>
+__device__ __forceinline__ auto pick(const P& t, int h) -> decltype(t.p[0]) {
+  auto r = t.p[0];
+#pragma unroll
+  for (int q = 1; q < kMaxEpRanks; ++q)
+    if (h == q) r = t.p[q];
+  return r;
+}
+
+// off[e] = rows of expert e that ranks 0..rank-1 send ahead of this rank's
+__device__ __forceinline__ void ep_offsets(const int32_t* __restrict__ cnt_all, int E, int rank,
+                                           int* off) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int o = 0;
+    for (int q = 0; q < rank; ++q) o += __ldg(cnt_all + static_cast<int64_t>(q) * E + e);
+    off[e] = o;
+  }
+}
+
+template <int K>
+__global__ void __launch_bounds__(256) ep_dispatch_kernel(
+    int64_t T, int row_vec, int E, int El, int rank, int world, int PC, const uint4* __restrict__ x,
+    const int32_t* __restrict__ expert_idx, const int32_t* __restrict__ slot,
+    const uint8_t* __restrict__ kept, const int32_t* __restrict__ cnt_all, PeerRows xe,
+    int32_t* __restrict__ local_cnt, int32_t* __restrict__ status) {
+  __shared__ int s_off[256];
+  dev::pdl_trigger();
+  dev::pdl_wait();
+  ep_offsets(cnt_all, E, rank, s_off);
+  // rows each of this rank's experts receives from all ranks (the FFN's counts)
+  if (blockIdx.x == 0 && local_cnt)
+    for (int el = threadIdx.x; el < El; el += blockDim.x) {
+      int n = 0;
+      for (int q = 0; q < world; ++q)
+        n += __ldg(cnt_all + static_cast<int64_t>(q) * E + static_cast<int64_t>(rank) * El + el);
+      local_cnt[el] = n;
+    }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  bool bad = false;
+  for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
+       t += nwarps) {
+    uint4* dst[K];
+    int nd = 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      if (!__ldg(kept + t * K + j)) continue;
+      const int e = __ldg(expert_idx + t * K + j);
+      const int64_t row = int64_t(e >= 0 && e < E ? s_off[e] : -1) + __ldg(slot + t * K + j);
+      if (e < 0 || e >= E || row < 0 || row >= PC) {  // counts that do not match the assignment
+        bad = true;
+        continue;
+      }
+      const int h = e / El;
+      dst[nd++] = pick(xe, h) + (static_cast<int64_t>(e - h * El) * PC + row) * row_vec;
+    }
+    if (nd == 0) continue;
+    const uint4* src = x + t * row_vec;
+#pragma unroll 4
+    for (int v = lane; v < row_vec; v += 32) {
+      const uint4 val = __ldg(src + v);
+      dst[0][v] = val;
+      if (K == 2 && nd == 2) dst[K - 1][v] = val;
+    }
+  }
+  // this thread's stores to peer memory are performed before the kernel ends
+  __threadfence_system();
+  if (bad && lane == 0 && status) atomicOr(status, MOE_STATUS_BAD_COUNTS);
+}
+
+template <int K, class V>
+__global__ void __launch_bounds__(256) ep_combine_kernel(
+    int64_t T, int row_vec, int E, int El, int rank, int PC, PeerRowsConst ye,
+    const int32_t* __restrict__ expert_idx, const float* __restrict__ gate,
+    const int32_t* __restrict__ slot, const uint8_t* __restrict__ kept,
+    const int32_t* __restrict__ cnt_all, uint4* __restrict__ y, int32_t* __restrict__ status) {
+  __shared__ int s_off[256];
+  dev::pdl_trigger();
+  dev::pdl_wait();
+  ep_offsets(cnt_all, E, rank, s_off);
+  __syncthreads();
+  constexpr int N = V::kN;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  bool bad = false;
+  for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
+       t += nwarps) {
+    const uint4* src[K];
+    float g[K];
+    int ns = 0;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      if (!__ldg(kept + t * K + j)) continue;
+      const int e = __ldg(expert_idx + t * K + j);
+      const int64_t row = int64_t(e >= 0 && e < E ? s_off[e] : -1) + __ldg(slot + t * K + j);
+      if (e < 0 || e >= E || row < 0 || row >= PC) {
+        bad = true;
+        continue;
+      }
+      const int h = e / El;
+      src[ns] = pick(ye, h) + (static_cast<int64_t>(e - h * El) * PC + row) * row_vec;
+      g[ns] = __ldg(gate + t * K + j);
+      ++ns;
+    }
+    uint4* dst = y + t * row_vec;
+#pragma unroll 2
+    for (int v = lane; v < row_vec; v += 32) {
+      float acc[N];
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] = 0.f;
+      if (ns > 0) {
+        const uint4 r0 = __ldg(src[0] + v);
+        uint4 r1 = make_uint4(0, 0, 0, 0);
+        if (K == 2 && ns == 2) r1 = __ldg(src[K - 1] + v);
+        float f[N];
+        V::unpack(r0, f);
+#pragma unroll
+        for (int i = 0; i < N; ++i) acc[i] = g[0] * f[i];
+        if (K == 2 && ns == 2) {
+          V::unpack(r1, f);
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[i] = fmaf(g[K - 1], f[i], acc[i]);
+        }
+      }
+      dst[v] = V::pack(acc);
+    }
+  }
+  if (bad && lane == 0 && status) atomicOr(status, MOE_STATUS_BAD_COUNTS);
+}
+
 }  // namespace
 
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
@@ -195,6 +349,57 @@ int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* exper
                                                     gate, slot, kept, yv);
   }
   return check_launch("combine_kernel");
+}
+
+int32_t launch_ep_dispatch(const moe_config& c, int rank, int world, const void* x,
+                           const int32_t* expert_idx, const int32_t* slot, const uint8_t* kept,
+                           const int32_t* cnt_all, void* const* xe_peers, int32_t* local_cnt,
+                           int32_t* status, cudaStream_t s) {
+  const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
+  const int El = c.E / world;
+  const int PC = world * c.capacity;
+  PeerRows xe{};
+  for (int q = 0; q < world && xe_peers; ++q) xe.p[q] = static_cast<uint4*>(xe_peers[q]);
+  // T = 0 still writes local_cnt (other ranks' rows arrive all the same)
+  const unsigned grid = grid_for_tokens(std::max<int64_t>(c.T, 1));
+  const uint4* xv = static_cast<const uint4*>(x);
+  if (c.k == 1)
+    launch_pdl(ep_dispatch_kernel<1>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El, rank,
+               world, PC, xv, expert_idx, slot, kept, cnt_all, xe, local_cnt, status);
+  else
+    launch_pdl(ep_dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El, rank,
+               world, PC, xv, expert_idx, slot, kept, cnt_all, xe, local_cnt, status);
+  return check_launch("ep_dispatch_kernel");
+}
+
+int32_t launch_ep_combine(const moe_config& c, int rank, int world, const void* const* ye_peers,
+                          const int32_t* expert_idx, const float* gate, const int32_t* slot,
+                          const uint8_t* kept, const int32_t* cnt_all, void* y, int32_t* status,
+                          cudaStream_t s) {
+  if (c.T == 0) return MOE_OK;
+  const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
+  const int El = c.E / world;
+  const int PC = world * c.capacity;
+  PeerRowsConst ye{};
+  for (int q = 0; q < world && ye_peers; ++q) ye.p[q] = static_cast<const uint4*>(ye_peers[q]);
+  const unsigned grid = grid_for_tokens(c.T);
+  uint4* yv = static_cast<uint4*>(y);
+  if (c.dtype == MOE_DTYPE_BF16) {
+    if (c.k == 1)
+      launch_pdl(ep_combine_kernel<1, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El,
+                 rank, PC, ye, expert_idx, gate, slot, kept, cnt_all, yv, status);
+    else
+      launch_pdl(ep_combine_kernel<2, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El,
+                 rank, PC, ye, expert_idx, gate, slot, kept, cnt_all, yv, status);
+  } else {
+    if (c.k == 1)
+      launch_pdl(ep_combine_kernel<1, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El,
+                 rank, PC, ye, expert_idx, gate, slot, kept, cnt_all, yv, status);
+    else
+      launch_pdl(ep_combine_kernel<2, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El,
+                 rank, PC, ye, expert_idx, gate, slot, kept, cnt_all, yv, status);
+  }
+  return check_launch("ep_combine_kernel");
 }
 
 }  // namespace moe

@@ -127,6 +127,46 @@ def test_calls_rejected_on_host(moe):
     assert moe.lib.moe_aux_loss(ctypes.byref(c), p, 0.01, p, None, None, p, ws - 1, None) == -4
 
 
+def test_expert_parallel_host_checks(moe):
+    """moe_ep_ffn_config derives the per-rank FFN config; the EP calls reject
+    bad rank/world, world not dividing E and unaligned or missing peer
+    pointers before any launch."""
+    c = cfg(moe)  # E = 128
+    out = moe.MoEConfig()
+    for world in (1, 2, 4, 8):
+        assert moe.lib.moe_ep_ffn_config(ctypes.byref(c), world, ctypes.byref(out)) == 0
+        assert (out.E, out.capacity) == (c.E // world, world * c.capacity)
+        assert (out.T, out.d_model, out.d_ff, out.dtype, out.expert) == \
+            (c.T, c.d_model, c.d_ff, c.dtype, c.expert)
+        assert (out.k, out.mode, out.num_groups) == (1, 0, 1)
+    for world in (0, 9, -1):
+        assert moe.lib.moe_ep_ffn_config(ctypes.byref(c), world, ctypes.byref(out)) == -1
+    c3 = cfg(moe, E=6)
+    assert moe.lib.moe_ep_ffn_config(ctypes.byref(c3), 4, ctypes.byref(out)) == -1
+    assert moe.lib.moe_ep_ffn_config(ctypes.byref(c), 2, None) == -1
+    # RRE layers keep their routing fields on the caller's side only
+    rre = cfg(moe, mode="rre", num_groups=4)
+    assert moe.lib.moe_ep_ffn_config(ctypes.byref(rre), 8, ctypes.byref(out)) == 0
+    assert (out.E, out.mode, out.num_groups) == (16, 0, 1)
+
+    p = ctypes.c_void_p(4096)
+    peers = (ctypes.c_void_p * 2)(4096, 8192)
+    bad_peers = (ctypes.c_void_p * 2)(4096, 8200)
+    null_peer = (ctypes.c_void_p * 2)(4096, None)
+    disp = moe.lib.moe_ep_dispatch
+    assert disp(ctypes.byref(c), 2, 2, p, p, p, p, p, peers, p, None, None) == -1   # rank >= world
+    assert disp(ctypes.byref(c), 0, 9, p, p, p, p, p, peers, p, None, None) == -1   # world > 8
+    assert disp(ctypes.byref(c3), 0, 4, p, p, p, p, p, peers, p, None, None) == -1  # 4 does not divide 6
+    assert disp(ctypes.byref(c), 0, 2, p, p, p, p, p, bad_peers, p, None, None) == -3
+    assert disp(ctypes.byref(c), 0, 2, p, p, p, p, p, null_peer, p, None, None) == -1
+    assert disp(ctypes.byref(c), 0, 2, p, p, p, p, p, None, p, None, None) == -1
+    assert disp(ctypes.byref(c), 0, 2, p, p, p, p, None, peers, p, None, None) == -1  # cnt_all
+    comb = moe.lib.moe_ep_combine
+    assert comb(ctypes.byref(c), 0, 2, peers, p, p, p, p, p, None, None, None) == -1   # y null
+    assert comb(ctypes.byref(c), 0, 2, bad_peers, p, p, p, p, p, p, None, None) == -3
+    assert comb(ctypes.byref(c), 3, 2, peers, p, p, p, p, p, p, None, None) == -1
+
+
 def test_library_refuses_cpu_tensors(moe):
     import torch
     c = cfg(moe, T=4, d_model=64, d_ff=64, E=16, capacity_=1)

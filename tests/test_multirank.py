@@ -55,3 +55,41 @@ def test_two_gloo_ranks_aggregate():
         assert tok == 128.0        # tokens of all ranks
         assert not same_x          # each rank has its own batch
         assert same_w              # experts are replicated
+
+
+def _ep_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from sparse_mixture_experts_fwd_b200.ep import exchange_counts, rank_barrier
+        E = 12
+        kept_cnt = (torch.arange(E, dtype=torch.int32) * (rank + 1)) % 7
+        out = torch.full((world, E), -1, dtype=torch.int32)
+        cnt_all = exchange_counts(kept_cnt, world, out=out)
+        token = torch.zeros(1, dtype=torch.int32)
+        rank_barrier(token)
+        q.put((rank, cnt_all.data_ptr() == out.data_ptr(), cnt_all.tolist(), int(token.item())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_count_exchange_gloo():
+    """The expert-parallel host plumbing on two gloo ranks: every rank gets
+    every rank's kept counts in rank order (in the caller's buffer), and the
+    barrier's token stays zero."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    want = [[(e * (r + 1)) % 7 for e in range(12)] for r in range(world)]
+    for rank, in_place, cnt_all, token in res:
+        assert in_place
+        assert cnt_all == want
+        assert token == 0
