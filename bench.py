@@ -491,6 +491,89 @@ def run_b200(args, w, world, rank, local):
         del gd, gs
         torch.cuda.empty_cache()
 
+    # ---- expert parallelism: two ranks emulated on this GPU ----
+    # Both ranks' receive buffers live on this device and each rank's peer
+    # table lists both, so the EP kernels issue the stores and loads they would
+    # send over NVLink, here against HBM.  Rank 0 routes this batch, rank 1
+    # the next rotated batch; the steps run in the order the cross-rank
+    # barriers impose (both dispatches, both expert FFNs, both combines).
+    ep = None
+    if world == 1 and w.E % 2 == 0:
+        P = 2
+        fcfg = moe.ep_ffn_config(cfg, P)
+        El, PC = fcfg.E, fcfg.capacity
+        rk = []
+        for q in range(P):
+            xq, dq = xs[q % n_rot], doms[q % n_rot]
+            if w.mode == "topk":
+                ro = moe.topk_assign(cfg, logits=moe.router(cfg, xq, Wr, bias, stream=stream),
+                                     stream=stream)
+            else:
+                ro = moe.topk_assign(cfg, domain_id=dq, stream=stream)
+            rk.append({"x": xq, "ro": ro,
+                       "xe": torch.empty(El, PC, w.d_model, dtype=w.torch_dtype, device=dev),
+                       "ye": torch.empty(El, PC, w.d_model, dtype=w.torch_dtype, device=dev),
+                       "H": torch.empty(El, PC, w.d_ff, dtype=w.torch_dtype, device=dev),
+                       "lc": torch.empty(El, dtype=torch.int32, device=dev),
+                       "y": torch.empty_like(y),
+                       "W1": W1[q * El:(q + 1) * El], "W2": W2[q * El:(q + 1) * El],
+                       "ws": torch.empty(max(256, moe.ffn_workspace_size(fcfg)),
+                                         dtype=torch.uint8, device=dev)})
+        with torch.cuda.stream(stream):
+            cnt_all = torch.stack([r["ro"]["kept_cnt"] for r in rk]).contiguous()
+        xe_peers = [r["xe"] for r in rk]
+        ye_peers = [r["ye"] for r in rk]
+        ep_status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def ep_step(evs):
+            evs[0].record(stream)
+            for q, r in enumerate(rk):
+                ro = r["ro"]
+                moe.ep_dispatch(cfg, q, P, r["x"], ro["expert_idx"], ro["slot"], ro["kept"],
+                                cnt_all, xe_peers, local_cnt=r["lc"], status=ep_status,
+                                stream=stream)
+            evs[1].record(stream)
+            for r in rk:
+                moe.expert_ffn(fcfg, r["xe"], r["W1"], r["W2"], r["lc"], H=r["H"], ye=r["ye"],
+                               workspace=r["ws"], status=ep_status, stream=stream)
+            evs[2].record(stream)
+            for q, r in enumerate(rk):
+                ro = r["ro"]
+                moe.ep_combine(cfg, q, P, ye_peers, ro["expert_idx"], ro["gate"], ro["slot"],
+                               ro["kept"], cnt_all, y=r["y"], status=ep_status, stream=stream)
+            evs[3].record(stream)
+
+        ep_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                  for _ in range(max(args.steps, args.warmup))]
+        for i in range(args.warmup):
+            ep_step(ep_evs[i])
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            ep_step(ep_evs[i])
+        torch.cuda.synchronize()
+        assert int(ep_status.item()) == 0, "expert-parallel step reported a device status"
+        t_d = sum(e[0].elapsed_time(e[1]) for e in ep_evs[:args.steps]) / args.steps
+        t_f = sum(e[1].elapsed_time(e[2]) for e in ep_evs[:args.steps]) / args.steps
+        t_c = sum(e[2].elapsed_time(e[3]) for e in ep_evs[:args.steps]) / args.steps
+        row = w.d_model * es
+        n_sent = sum(int(r["ro"]["kept"].sum()) for r in rk)
+        n_src = sum(int((r["ro"]["kept"].sum(1) > 0).sum()) for r in rk)
+        d_bytes = (n_src + n_sent) * row
+        c_bytes = (n_sent + P * w.T) * row
+        hbm = peaks["hbm_gbs"] * 1e9
+        ep = {"world": P, "tokens_per_step": P * w.T, "ffn_capacity": PC,
+              "dispatch_ms": t_d, "dispatch_bytes": d_bytes,
+              "dispatch_frac_hbm": d_bytes / hbm / (t_d / 1e3),
+              "expert_ffn_ms": t_f, "combine_ms": t_c, "combine_bytes": c_bytes,
+              "combine_frac_hbm": c_bytes / hbm / (t_c / 1e3),
+              "step_ms": t_d + t_f + t_c,
+              "tokens_per_s": P * w.T / ((t_d + t_f + t_c) / 1e3),
+              "note": "moe_ep_dispatch / moe_expert_ffn / moe_ep_combine for two ranks emulated "
+                      "on one GPU (peer stores and loads hit HBM, not NVLink); events between "
+                      "the three steps, routing outside the timed region"}
+        del rk, xe_peers, ye_peers
+        torch.cuda.empty_cache()
+
     # ---- e2e through moe_layer_forward with host buffers ----
     # Every step copies its batch from pinned host memory and its output back.
     # The copies run on two copy streams, double-buffered, so step i's
@@ -582,6 +665,7 @@ def run_b200(args, w, world, rank, local):
         "combine": "fused into the expert FFN's GEMM-2 epilogue" if fused_combine else "kernel",
         "aux_loss": aux,
         "sparseclip": sclip,
+        "expert_parallel": ep,
         "routing": {"n_kept": n_kept, "n_dropped": n_dropped,
                     "drop_rate": n_dropped / (w.T * w.k)},
         "gpu_launches": launches_per_step * args.steps,

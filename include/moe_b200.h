@@ -334,7 +334,10 @@ int32_t moe_ep_ffn_config(const moe_config* cfg, int32_t world, moe_config* out)
  * rank's own), each 16-byte aligned.  local_cnt [El] int32 (device,
  * nullable): receives sum over q of cnt_all[q, rank*El + el], the kept counts
  * for step 5.  A row whose index would fall outside 0..world*C-1 is skipped
- * and sets MOE_STATUS_BAD_COUNTS.  x [T, d] in cfg->dtype. */
+ * and sets MOE_STATUS_BAD_COUNTS.  x [T, d] in cfg->dtype.  Two launches: the
+ * copy, then a one-thread kernel whose system-scope fence makes the copy's
+ * stores visible to every device before the caller's next operation on
+ * `stream` (the barrier of step 4). */
 int32_t moe_ep_dispatch(const moe_config* cfg, int32_t rank, int32_t world, const void* x,
                         const int32_t* expert_idx, const int32_t* slot, const uint8_t* kept,
                         const int32_t* cnt_all, void* const* xe_peers, int32_t* local_cnt,

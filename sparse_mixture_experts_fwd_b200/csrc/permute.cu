@@ -47,13 +47,16 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
     for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0u;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
        t += nwarps) {
-    int64_t dst[K];
+    int64_t dst0 = 0, dst1 = 0;  // the kept choices' xe rows, in choice order
     int nd = 0;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
       if (__ldg(kept + t * K + j)) {
-        dst[nd++] = (static_cast<int64_t>(__ldg(expert_idx + t * K + j)) * C +
-                     __ldg(slot + t * K + j)) * row_vec;
+        const int64_t d = (static_cast<int64_t>(__ldg(expert_idx + t * K + j)) * C +
+                           __ldg(slot + t * K + j)) * row_vec;
+        if (nd == 0) dst0 = d;
+        else dst1 = d;
+        ++nd;
       }
     }
     if (nd == 0) {
@@ -67,8 +70,8 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
 #pragma unroll 4
     for (int v = lane; v < row_vec; v += 32) {
       const uint4 val = __ldg(src + v);
-      xe[dst[0] + v] = val;
-      if (K == 2 && nd == 2) xe[dst[K - 1] + v] = val;
+      xe[dst0 + v] = val;
+      if (K == 2 && nd == 2) xe[dst1 + v] = val;
     }
   }
 }
@@ -217,7 +220,8 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(
   bool bad = false;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
        t += nwarps) {
-    uint4* dst[K];
+    uint4* dst0 = nullptr;  // the kept choices' destination rows, in choice order
+    uint4* dst1 = nullptr;
     int nd = 0;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
@@ -229,20 +233,34 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(
         continue;
       }
       const int h = e / El;
-      dst[nd++] = pick(xe, h) + (static_cast<int64_t>(e - h * El) * PC + row) * row_vec;
+      uint4* d = pick(xe, h) + (static_cast<int64_t>(e - h * El) * PC + row) * row_vec;
+      if (nd == 0) dst0 = d;
+      else dst1 = d;
+      ++nd;
     }
     if (nd == 0) continue;
     const uint4* src = x + t * row_vec;
 #pragma unroll 4
     for (int v = lane; v < row_vec; v += 32) {
       const uint4 val = __ldg(src + v);
-      dst[0][v] = val;
-      if (K == 2 && nd == 2) dst[K - 1][v] = val;
+      dst0[v] = val;
+      if (K == 2 && nd == 2) dst1[v] = val;
     }
   }
-  // this thread's stores to peer memory are performed before the kernel ends
-  __threadfence_system();
   if (bad && lane == 0 && status) atomicOr(status, MOE_STATUS_BAD_COUNTS);
+}
+
+// Runs after ep_dispatch_kernel on the same stream: griddepcontrol.wait
+// returns once the dispatch grid has completed and its stores are visible to
+// this grid, and the system-scope fence (cumulative over what this thread has
+// observed) then makes them visible to every device before the caller's next
+// operation, the cross-rank barrier.  One fence per dispatch instead of one
+// per warp, which would hold every warp of the copy until its peer stores are
+// acknowledged.
+__global__ void __launch_bounds__(32) ep_release_kernel() {
+  dev::pdl_trigger();
+  dev::pdl_wait();
+  if (threadIdx.x == 0) __threadfence_system();
 }
 
 template <int K, class V>
@@ -262,8 +280,9 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(
   bool bad = false;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
        t += nwarps) {
-    const uint4* src[K];
-    float g[K];
+    const uint4* src0 = nullptr;  // the kept choices' rows and gates, in choice order
+    const uint4* src1 = nullptr;
+    float g0 = 0.f, g1 = 0.f;
     int ns = 0;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
@@ -275,8 +294,15 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(
         continue;
       }
       const int h = e / El;
-      src[ns] = pick(ye, h) + (static_cast<int64_t>(e - h * El) * PC + row) * row_vec;
-      g[ns] = __ldg(gate + t * K + j);
+      const uint4* r = pick(ye, h) + (static_cast<int64_t>(e - h * El) * PC + row) * row_vec;
+      const float gj = __ldg(gate + t * K + j);
+      if (ns == 0) {
+        src0 = r;
+        g0 = gj;
+      } else {
+        src1 = r;
+        g1 = gj;
+      }
       ++ns;
     }
     uint4* dst = y + t * row_vec;
@@ -286,17 +312,17 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(
 #pragma unroll
       for (int i = 0; i < N; ++i) acc[i] = 0.f;
       if (ns > 0) {
-        const uint4 r0 = __ldg(src[0] + v);
+        const uint4 r0 = __ldg(src0 + v);
         uint4 r1 = make_uint4(0, 0, 0, 0);
-        if (K == 2 && ns == 2) r1 = __ldg(src[K - 1] + v);
+        if (K == 2 && ns == 2) r1 = __ldg(src1 + v);
         float f[N];
         V::unpack(r0, f);
 #pragma unroll
-        for (int i = 0; i < N; ++i) acc[i] = g[0] * f[i];
+        for (int i = 0; i < N; ++i) acc[i] = g0 * f[i];
         if (K == 2 && ns == 2) {
           V::unpack(r1, f);
 #pragma unroll
-          for (int i = 0; i < N; ++i) acc[i] = fmaf(g[K - 1], f[i], acc[i]);
+          for (int i = 0; i < N; ++i) acc[i] = fmaf(g1, f[i], acc[i]);
         }
       }
       dst[v] = V::pack(acc);
@@ -369,7 +395,10 @@ int32_t launch_ep_dispatch(const moe_config& c, int rank, int world, const void*
   else
     launch_pdl(ep_dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, El, rank,
                world, PC, xv, expert_idx, slot, kept, cnt_all, xe, local_cnt, status);
-  return check_launch("ep_dispatch_kernel");
+  const int32_t rc = check_launch("ep_dispatch_kernel");
+  if (rc != MOE_OK) return rc;
+  launch_pdl(ep_release_kernel, dim3(1), dim3(32), 0, s);
+  return check_launch("ep_release_kernel");
 }
 
 int32_t launch_ep_combine(const moe_config& c, int rank, int world, const void* const* ye_peers,
