@@ -19,9 +19,11 @@
 // of q''s kept count of e, in q's slot (token) order.  ep_dispatch_kernel
 // stores each kept row straight into the home rank's buffer through its peer
 // mapping (NVLink stores; a plain store when h is this rank), and
-// ep_combine_kernel loads each token's expert outputs back the same way.
-// Neither waits on another rank: the caller orders dispatch -> expert FFN ->
-// combine across ranks (a collective between the steps).
+// ep_combine_kernel loads each token's expert outputs back the same way.  A
+// one-thread ep_release_kernel after the dispatch issues the single
+// system-scope fence that publishes the copy's peer stores.  None of them
+// waits on another rank: the caller orders dispatch -> expert FFN -> combine
+// across ranks (a collective between the steps).
 #include <algorithm>
 
 #include "moe_internal.cuh"
