@@ -37,8 +37,8 @@ L2_BYTES = 126 * 1024 * 1024
 # capture of the kernels as shipped (the profile named beside each number).
 # A workload without a capture of its current kernels reports null.
 FFN_TRAFFIC = {
-    "switch_base": (1242.1e6 + 29.3e6, "profiles/ffn_tc_switch_base.md"),
-    "xmoe_top2": (604.1e6 + 227.9e6 + 825.7e6 + 59.5e6, "profiles/gemm_pair_xmoe_top2.md"),
+    "switch_base": (1240.836e6 + 29.177e6, "profiles/ffn_tc_switch_base.md"),
+    "xmoe_top2": (604.122e6 + 228.916e6 + 825.805e6 + 55.799e6, "profiles/gemm_pair_xmoe_top2.md"),
 }
 METRIC = "MoE-layer tokens/sec (1 B200); expert-FFN TFLOP/s; dispatch+combine GB/s"
 
