@@ -14,11 +14,12 @@
 // Roles: in each CTA warp 0 lane 0 loads its halves with TMA; the loads of
 // both CTAs complete on CTA 0's "full" barrier, which CTA 0 arms with the
 // pair's byte count.  CTA 0's warp 1 lane 0 issues the MMAs and commits them
-// with a multicast arrive on both CTAs' "empty" (stage free) and "tfull"
-// (accumulator ready) barriers.  Warps 2-5 of each CTA drain their own TMEM
-// and arrive on CTA 0's "tempty" barrier (remotely from CTA 1).  Every wait is
-// bounded; a cluster barrier brackets the kernel so neither CTA frees TMEM or
-// exits while the other still uses it.  No load uses cluster multicast.
+// with one tcgen05.commit that arrives on both CTAs' "empty" (stage free) and
+// "tfull" (accumulator ready) barriers.  Warps 2-5 of each CTA drain their own
+// TMEM and arrive on CTA 0's "tempty" barrier (remotely from CTA 1).  Every
+// wait is bounded; a cluster barrier brackets the kernel so neither CTA frees
+// TMEM or exits while the other still uses it.  Each CTA's TMA loads fill only
+// its own shared memory.
 #include <cuda.h>
 
 #include <algorithm>

@@ -189,7 +189,7 @@ MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int3
   }
 }
 
-// -- TMA (no multicast anywhere in this library) --
+// -- TMA (every load fills the issuing CTA's own shared memory) --
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
