@@ -167,6 +167,31 @@ def test_expert_parallel_host_checks(moe):
     assert comb(ctypes.byref(c), 3, 2, peers, p, p, p, p, p, p, None, None) == -1
 
 
+def test_expert_parallel_binding_host_side(moe):
+    """The Python side of the EP calls: the peer table, the per-rank FFN config
+    and the refusal of CPU tensors, all before any CUDA call."""
+    import torch
+    t = moe._peer_table([4096, 8192], 2, "xe_peers")
+    assert list(t) == [4096, 8192]
+    assert moe._peer_table(None, 2, "xe_peers") is None
+    with pytest.raises(ValueError, match="needs 2 entries"):
+        moe._peer_table([4096], 2, "xe_peers")
+    c = cfg(moe, T=4, d_model=64, d_ff=64, E=4, capacity_=2)
+    f = moe.ep_ffn_config(c, 2)
+    assert (f.E, f.capacity, f.T, f.d_model) == (2, 4, 4, 64)
+    with pytest.raises(moe.MoEError, match="does not divide"):
+        moe.ep_ffn_config(c, 3)
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    idx = torch.zeros(4, 1, dtype=torch.int32)
+    cnt = torch.zeros(2, 4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        moe.ep_dispatch(c, 0, 2, x, idx, idx, idx.to(torch.uint8), cnt, [4096, 8192],
+                        local_cnt=torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        moe.ep_combine(c, 0, 2, [4096, 8192], idx, torch.ones(4, 1), idx, idx.to(torch.uint8),
+                       cnt, y=x)
+
+
 def test_library_refuses_cpu_tensors(moe):
     import torch
     c = cfg(moe, T=4, d_model=64, d_ff=64, E=16, capacity_=1)
