@@ -7,6 +7,10 @@ this package; the CUDA library never calls it and shares no code with it.
 
 All array arguments are CPU torch tensors; activation tensors are bf16 or
 fp32 (their raw bits are handed over unchanged).
+
+``MOE_ORACLE_LIB`` (environment): load that library instead of building
+``libmoe_oracle.so`` — the mutation test points the pin suite at copies of
+the oracle with one planted mistake each.
 """
 from __future__ import annotations
 
@@ -36,7 +40,7 @@ def _load():
     global _lib
     if _lib is not None:
         return _lib
-    lib = ctypes.CDLL(build())
+    lib = ctypes.CDLL(os.environ.get("MOE_ORACLE_LIB") or build())
     i64, i32, u64, dbl, vp = (ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64, ctypes.c_double,
                               ctypes.c_void_p)
     sig = {
