@@ -9,6 +9,7 @@ suite in the regular run.  CPU only.
 """
 import concurrent.futures as cf
 import os
+import shutil
 import subprocess
 import sys
 
@@ -112,10 +113,13 @@ def _run_mutant(name, edits, tmp):
     return r.returncode, r.stdout[-2000:]
 
 
-def test_every_planted_mistake_fails_a_pin(tmp_path):
+def test_every_planted_mistake_fails_a_pin():
+    tmp = os.path.join(ROOT, "_build", "oracle_mutants")  # a build folder, kept out of git
+    shutil.rmtree(tmp, ignore_errors=True)
+    os.makedirs(tmp)
     workers = max(1, min(8, (os.cpu_count() or 2) // 2))
     with cf.ThreadPoolExecutor(workers) as ex:
-        futs = {n: ex.submit(_run_mutant, n, e, str(tmp_path)) for n, e in MUTANTS.items()}
+        futs = {n: ex.submit(_run_mutant, n, e, tmp) for n, e in MUTANTS.items()}
         results = {n: f.result() for n, f in futs.items()}
     survivors = {n: out for n, (rc, out) in results.items() if rc == 0}
     assert not survivors, "mutants that pass every pin:\n" + "\n".join(
