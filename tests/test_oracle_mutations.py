@@ -121,6 +121,7 @@ def test_every_planted_mistake_fails_a_pin():
     with cf.ThreadPoolExecutor(workers) as ex:
         futs = {n: ex.submit(_run_mutant, n, e, tmp) for n, e in MUTANTS.items()}
         results = {n: f.result() for n, f in futs.items()}
+    shutil.rmtree(tmp, ignore_errors=True)
     survivors = {n: out for n, (rc, out) in results.items() if rc == 0}
     assert not survivors, "mutants that pass every pin:\n" + "\n".join(
         f"--- {n}\n{out}" for n, out in survivors.items())
