@@ -160,13 +160,13 @@ def sum_over_ranks(v: float, world: int, device: str = "cuda") -> float:
 # CPU oracle timing (the reference arm and the cpu_baseline object)
 # ---------------------------------------------------------------------------
 
-def oracle_step_fn(w, T_s):
+def oracle_step_fn(w, T_s, threads=None):
     """A closure running the oracle's whole layer on the first T_s tokens of the workload."""
     import oracle
     ws = w.scaled(T=T_s)
     inp = synth.layer_inputs(ws)
     C = oracle.capacity(ws.T, ws.E, ws.capacity_factor)
-    nth = os.cpu_count() or 1
+    nth = threads or os.cpu_count() or 1
 
     def step():
         oracle.layer_forward(inp["x"], inp["W1"], inp["W2"], E=ws.E, k=ws.k, C=C, Wr=inp["Wr"],
@@ -191,9 +191,19 @@ def cpu_baseline(w, seconds):
     t0 = time.perf_counter()
     step()
     dt = time.perf_counter() - t0
+    # the same oracle on one thread, on a sample sized from the multithreaded
+    # rate for about a quarter of `seconds`
+    T_1 = max(16, min(T_s, int(T_s / max(dt, 1e-6) / nth * seconds / 4)))
+    step1, _ = oracle_step_fn(w, T_1, threads=1)
+    t1 = time.perf_counter()
+    step1()
+    dt1 = time.perf_counter() - t1
     return {"value": T_s / dt, "unit": "tokens/s", "cores": nth, "kind": "oracle",
             "sample": f"whole layer on the first {T_s} of {w.T} tokens (capacity from eq. 3 at "
-                      f"T={T_s}), fp64 CPU oracle, {nth} threads, one timed pass of {dt:.2f} s"}
+                      f"T={T_s}), fp64 CPU oracle, {nth} threads, one timed pass of {dt:.2f} s",
+            "value_1thread": T_1 / dt1,
+            "sample_1thread": f"whole layer on the first {T_1} tokens (capacity from eq. 3 at "
+                              f"T={T_1}), 1 thread, {dt1:.2f} s"}
 
 
 def run_reference(args, w, world, rank):
