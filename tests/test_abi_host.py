@@ -199,3 +199,59 @@ def test_library_refuses_cpu_tensors(moe):
     with pytest.raises(ValueError, match="CUDA"):
         moe.router(c, x, torch.zeros(16, 64, dtype=torch.bfloat16),
                    logits=torch.zeros(4, 16))
+
+
+def _expected_check(T, d, f, E, k, C, mode, G, dtype, expert):
+    """The documented validity rules of moe_config, restated (header and DESIGN)."""
+    I32 = 2 ** 31 - 1
+    if T < 0 or T > I32 or E < 1:
+        return -1
+    if E > 256 or k not in (1, 2):
+        return -2
+    if k > E or C < 0:
+        return -1
+    if mode == 1 and (k != 1 or G < 1 or E % G):
+        return -1
+    if expert == 1 and dtype != 0:
+        return -2
+    if d < 1 or f < 1:
+        return -1
+    if (dtype == 0 and (d % 64 or f % 64)) or (dtype == 1 and (d % 4 or f % 4)):
+        return -2
+    if E * C > I32 or E * f * 2 > I32 or E * d > I32:
+        return -2
+    return 0
+
+
+def test_config_check_property(moe):
+    """moe_config_check agrees with the documented rules on random configs, and
+    every accepted config gets an ordered, 256-byte aligned workspace layout."""
+    hyp = pytest.importorskip("hypothesis")
+    st = hyp.strategies
+
+    @hyp.settings(max_examples=400, deadline=None, derandomize=True)
+    @hyp.given(T=st.integers(-3, 3 * 2 ** 20), d=st.sampled_from([0, 4, 32, 64, 100, 128, 768]),
+               f=st.sampled_from([0, 4, 48, 64, 96, 256, 3072]), E=st.integers(-1, 300),
+               k=st.integers(0, 3), C=st.integers(-2, 5000), mode=st.integers(0, 1),
+               G=st.integers(0, 9), dtype=st.integers(0, 1), expert=st.integers(0, 1))
+    def check(T, d, f, E, k, C, mode, G, dtype, expert):
+        c = moe.MoEConfig(T=T, d_model=d, d_ff=f, E=E, k=k, capacity=C, mode=mode, num_groups=G,
+                          dtype=dtype, expert=expert, reserved=0, seed=1)
+        want = _expected_check(T, d, f, E, k, C, mode, G, dtype, expert)
+        assert moe.lib.moe_config_check(ctypes.byref(c)) == want
+        if want != 0:
+            assert moe.lib.moe_workspace_size(ctypes.byref(c)) == 0
+            return
+        m = moe.workspace_layout(c)
+        es = 2 if dtype == 0 else 4
+        offs = [m.logits, m.expert_idx, m.gate, m.slot, m.kept, m.tok_of_row, m.arrivals,
+                m.kept_cnt, m.n_dropped, m.scratch, m.ffn_sync, m.xe, m.H, m.ye, m.total]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert m.expert_idx - m.logits >= (T * E * 4 if (mode == 0 and dtype == 1) else 0)
+        assert m.gate - m.expert_idx >= T * k * 4 and m.kept_cnt - m.arrivals >= E * 4
+        assert m.tok_of_row - m.kept >= T * k and m.arrivals - m.tok_of_row >= E * C * 4
+        assert m.H - m.xe >= E * C * d * es and m.ye - m.H >= E * C * f * es
+        assert m.total - m.ye >= E * C * d * es
+        assert moe.lib.moe_workspace_size(ctypes.byref(c)) == m.total
+
+    check()
