@@ -48,7 +48,10 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="switch_base", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="pangu_rre", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling captures: the workload cut to this many experts with the "
+                         "same tokens per expert (T scaled by E'/E, same capacity)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--expert", default="relu", choices=["relu", "geglu"],
                     help="expert network (the workloads are defined with the ReLU FFN)")
@@ -245,7 +248,9 @@ def kernel_launches(w, C):
         route = 2                       # router GEMM with gate/top-k epilogue, slot assignment
     else:
         route = 3                       # fp32 router, gate/top-k, slot assignment
-    ffn = 1 if (bf16 and C <= 128) else 2
+    # bf16: one persistent kernel for both GEMMs when C <= 128 (single CTAs) or
+    # C >= 512 (SM pairs); two grouped launches in between; fp32: two FMA GEMMs
+    ffn = 1 if (bf16 and (C <= 128 or C >= 512)) else 2
     combine = 0 if (bf16 and w.k == 1) else 1   # top-1 bf16: inside the FFN's GEMM 2
     return route + 1 + ffn + combine
 
@@ -424,7 +429,7 @@ def run_b200(args, w, world, rank, local):
         "grouped_gemm_f32_kernel x2" if w.dtype == "f32" else
         "ffn_tc_kernel x1 (both GEMMs fused)" if C <= 128 else
         "gemm_tc_kernel x2 (H = ReLU(xe W1^T), ye = H W2^T)" if C < 512 else
-        "gemm_pair_kernel x2 on SM pairs (H = ReLU(xe W1^T), ye = H W2^T)"))
+        "ffn_pair_kernel x1 on SM pairs (both GEMMs fused, tokens on the MMA's N side)"))
     roof["peak_source"] = peaks["source"]
     roof["algorithmic_per_launch"] = (f"{ffn_bytes / 1e9:.4f} GB" if roof["bound"] == "hbm"
                                       else f"{ffn_flops / 1e12:.4f} TFLOP")
@@ -692,6 +697,11 @@ def run_b200(args, w, world, rank, local):
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
+    if args.experts:
+        if args.experts <= 0 or w.E % args.experts or args.experts % max(1, w.num_groups):
+            raise SystemExit("--experts must divide E and be a multiple of the group count")
+        w = w.scaled(name=f"{w.name}_E{args.experts}", E=args.experts,
+                     T=w.T * args.experts // w.E)
     if args.expert != "relu":
         w = w.scaled(expert=args.expert)
     world, rank, local = (1, 0, 0)

@@ -32,6 +32,14 @@
  *   * Conditions seen on the device are OR-ed into the optional `status`
  *     word (device int32, nullable; enum moe_status_bits).  The caller
  *     zeroes `status` before the call and reads it after synchronising.
+ *   * Every wait inside a kernel is bounded (1 s by default, see
+ *     moe_set_wait_limit_ns).  The status word is also the call's give-up
+ *     signal: once one wait expires and sets MOE_STATUS_TIMEOUT, every other
+ *     wait of every kernel that shares the word gives up at its next poll, so
+ *     the whole call ends within about one limit.  A call that starts with
+ *     the timeout bit already set therefore gives up its waits at once (its
+ *     outputs are invalid, as the bit says).  Without a status word each
+ *     thread block gives up on its own limit.
  */
 #ifndef MOE_B200_H_
 #define MOE_B200_H_
@@ -65,7 +73,7 @@ enum moe_route_mode { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RRE = 1 };
  * with GELU(a) = a * Phi(a) (the erf form), out = H W2^T; bf16 layers only. */
 enum moe_expert { MOE_EXPERT_RELU = 0, MOE_EXPERT_GEGLU = 1 };
 enum moe_status_bits {
-  MOE_STATUS_TIMEOUT = 1,   /* a pipeline wait gave up after 1 s; outputs invalid     */
+  MOE_STATUS_TIMEOUT = 1,   /* a pipeline wait gave up (wait limit); outputs invalid  */
   MOE_STATUS_BAD_DOMAIN = 2, /* an RRE domain id was outside 0..G-1 (routed as 0)      */
   MOE_STATUS_BAD_COUNTS = 4  /* expert parallel: a row fell outside its expert's block
                                 (counts that do not match the assignment); skipped     */
@@ -120,6 +128,15 @@ size_t moe_workspace_map_size(void);
 const char* moe_error_string(int32_t code);
 /* Detail of the last error returned on the calling host thread ("" if none). */
 const char* moe_last_error(void);
+
+/* Limit of every bounded wait inside the library's kernels, in ns, for the
+ * launches made after this call by any host thread (process-wide); 0
+ * restores the default of 1 s.  For tests of the failure path and for
+ * debugging: a wait that can never be met then ends within this limit and
+ * the call reports MOE_STATUS_TIMEOUT.  moe_wait_limit_ns returns the value
+ * in force. */
+void moe_set_wait_limit_ns(uint64_t ns);
+uint64_t moe_wait_limit_ns(void);
 
 /* Eq. (3) of the Switch notes, sec. 2.2: floor(T / E * capacity_factor).
  * Returns -1 if E < 1, T < 0 or capacity_factor < 0. */
@@ -189,13 +206,37 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert
  * round(GELU(xe[e, r, :] . W1[e, 2i]) * (xe[e, r, :] . W1[e, 2i + 1])))
  * for r < kept_cnt[e] (device int32 [E], values in 0..C).  xe, ye
  * [E, C, d] and H [E, C, f] (caller-provided scratch) in cfg->dtype; other
- * rows of H and ye are left untouched.  bf16: one persistent tcgen05 kernel
- * runs both GEMMs with fp32 accumulation; workspace holds its tile counters
- * (moe_ffn_workspace_size bytes, zeroed by the call; unused for fp32, which
- * runs FMA GEMMs and may pass null). */
+ * rows of H and ye are left untouched.  bf16 runs tcgen05 kernels with fp32
+ * accumulation, chosen by the capacity: C <= 128, one persistent kernel for
+ * both GEMMs (128 x 256 tiles); 128 < C < 512, two grouped launches (one per
+ * GEMM, 128 x 256 tiles); C >= 512, two grouped launches on SM pairs
+ * (256 x 256 tiles, cta_group::2).  workspace: moe_ffn_workspace_size bytes
+ * (zeroed by the call; the persistent kernel's tile counters).  fp32 runs
+ * FMA GEMMs and may pass a null workspace. */
 int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
                        const int32_t* kept_cnt, void* H, void* ye, void* workspace,
                        size_t workspace_bytes, int32_t* status, moe_stream_t stream);
+
+/* Flags of moe_expert_ffn_ex. */
+enum moe_ffn_flags {
+  /* The caller has already zeroed the workspace's moe_ffn_workspace_size
+   * bytes earlier on `stream` (for example inside a kernel of its own), so
+   * the call launches no memset and the persistent kernel reads its counters
+   * as it finds them.  Its counters (uint32): word 0 numbers the tiles as
+   * thread blocks take them; word 1 + e * ceil(C / 256) + c counts the
+   * finished GEMM-1 work of rows chunk c of expert e (chunks of at most 256
+   * rows; c = 0 when C <= 256), and the GEMM-2 tiles of that chunk wait
+   * (bounded) until the count minus its total, as a signed 32-bit
+   * difference, is >= 0.  A word preset to -n therefore ends n short and
+   * that wait runs out. */
+  MOE_FFN_WORKSPACE_ZEROED = 1
+};
+
+/* moe_expert_ffn with flags (enum moe_ffn_flags; 0 = moe_expert_ffn). */
+int32_t moe_expert_ffn_ex(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
+                          const int32_t* kept_cnt, void* H, void* ye, void* workspace,
+                          size_t workspace_bytes, uint32_t flags, int32_t* status,
+                          moe_stream_t stream);
 
 /* Combine (Switch notes sec. 2.1, eq. 2; drop rule sec. 2.2):
  *   y[t, :] = sum over kept j of gate[t, j] * ye[expert_idx[t, j], slot[t, j], :]
@@ -277,9 +318,10 @@ int32_t sparseclip_clip(float* const* dense, const int64_t* dense_len, int32_t n
  * device memory, present on every GPU that loads the library until the
  * process exits.  Limits and behaviour:
  *   * n_dense + n_sparse <= 1024, else MOE_ERR_UNSUPPORTED (nothing launched);
- *   * the first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture;
+ *   * the first call with a device (and CUDA context) current looks up the
+ *     array's device address and caches it per device and context, so a
+ *     caller that switches contexts or resets the device gets a fresh
+ *     lookup; make that first call before any stream capture;
  *   * the call allocates nothing (no cudaMalloc/cudaFree, no allocating
  *     library routine);
  *   * every call on a device shares the array: calls that overlap on the

@@ -21,7 +21,7 @@
 //     experts grouped by domain, each token sent uniformly at random to an
 //     expert of its domain's group through an unweighted gate.
 //
-// Readings where the pages are silent (each one is listed in the design doc):
+// Readings taken where the pages are silent:
 //   * capacity: C = floor(T * capacity_factor / E), passed on as an integer;
 //   * top-k is taken on the fp32 logits (softmax is monotone), ties go to
 //     the lowest expert index; the k gates are the raw softmax values of

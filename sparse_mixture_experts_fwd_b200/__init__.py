@@ -24,6 +24,7 @@ ERRORS = {-1: "MOE_ERR_INVALID_ARGUMENT", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ER
 DTYPE_BF16, DTYPE_F32 = 0, 1
 ROUTE_TOPK, ROUTE_RRE = 0, 1
 STATUS_TIMEOUT, STATUS_BAD_DOMAIN, STATUS_BAD_COUNTS = 1, 2, 4
+FFN_WORKSPACE_ZEROED = 1
 
 # every entry point the header declares, with its ctypes signature
 _i32, _i64, _u64, _sz, _vp, _dbl = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64,
@@ -65,6 +66,10 @@ SIGNATURES = {
     "moe_dispatch": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "moe_ffn_workspace_size": ([_PCFG], _sz),
     "moe_expert_ffn": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp], _i32),
+    "moe_expert_ffn_ex": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, ctypes.c_uint32, _vp,
+                           _vp], _i32),
+    "moe_set_wait_limit_ns": ([_u64], None),
+    "moe_wait_limit_ns": ([], _u64),
     "moe_combine": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "moe_layer_forward": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp],
                           _i32),
@@ -240,8 +245,18 @@ def ffn_workspace_size(cfg: MoEConfig) -> int:
     return int(lib.moe_ffn_workspace_size(ctypes.byref(cfg)))
 
 
+def set_wait_limit_ns(ns: int):
+    """Limit of every bounded wait in the library's kernels (0 = the 1 s default)."""
+    lib.moe_set_wait_limit_ns(int(ns))
+
+
+def wait_limit_ns() -> int:
+    return int(lib.moe_wait_limit_ns())
+
+
 def expert_ffn(cfg, xe, W1, W2, kept_cnt, H=None, ye=None, workspace=None, status=None,
-               stream=None):
+               stream=None, flags=0):
+    """flags: FFN_WORKSPACE_ZEROED = the caller zeroed ``workspace`` on the stream already."""
     if H is None:
         H = torch.empty(cfg.E, cfg.capacity, cfg.d_ff, dtype=xe.dtype, device=xe.device)
     if ye is None:
@@ -249,10 +264,11 @@ def expert_ffn(cfg, xe, W1, W2, kept_cnt, H=None, ye=None, workspace=None, statu
     if workspace is None:
         workspace = torch.empty(max(256, ffn_workspace_size(cfg)), dtype=torch.uint8,
                                 device=xe.device)
-    _check(lib.moe_expert_ffn(ctypes.byref(cfg), _ptr(xe, "xe"), _ptr(W1, "W1"), _ptr(W2, "W2"),
-                              _ptr(kept_cnt, "kept_cnt"), _ptr(H, "H"), _ptr(ye, "ye"),
-                              _ptr(workspace, "workspace"), workspace.numel(),
-                              _ptr(status, "status"), _stream(stream)), "moe_expert_ffn")
+    _check(lib.moe_expert_ffn_ex(ctypes.byref(cfg), _ptr(xe, "xe"), _ptr(W1, "W1"),
+                                 _ptr(W2, "W2"), _ptr(kept_cnt, "kept_cnt"), _ptr(H, "H"),
+                                 _ptr(ye, "ye"), _ptr(workspace, "workspace"), workspace.numel(),
+                                 int(flags), _ptr(status, "status"), _stream(stream)),
+           "moe_expert_ffn_ex")
     return H, ye
 
 

@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation, workspace layout and the layer
 // forward sequence.  Every device-side step is one of the library's kernels.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <string>
@@ -11,7 +12,10 @@ namespace moe {
 
 namespace {
 thread_local std::string g_last_error;
+std::atomic<uint64_t> g_wait_limit_ns{dev::kDefaultWaitLimitNs};
 }
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 void set_last_error(const std::string& msg) { g_last_error = msg; }
 
@@ -157,6 +161,12 @@ const char* moe_error_string(int32_t code) {
 
 const char* moe_last_error(void) { return last_error_cstr(); }
 
+void moe_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? dev::kDefaultWaitLimitNs : ns, std::memory_order_relaxed);
+}
+
+uint64_t moe_wait_limit_ns(void) { return wait_limit_ns(); }
+
 int32_t moe_capacity(int64_t T, int32_t E, double capacity_factor) {
   if (E < 1 || T < 0 || !(capacity_factor >= 0.0)) return -1;
   const double c = std::floor(static_cast<double>(T) / E * capacity_factor);
@@ -252,7 +262,17 @@ size_t moe_ffn_workspace_size(const moe_config* cfg) {
 int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
                        const int32_t* kept_cnt, void* H, void* ye, void* workspace,
                        size_t workspace_bytes, int32_t* status, moe_stream_t stream) {
+  return moe_expert_ffn_ex(cfg, xe, W1, W2, kept_cnt, H, ye, workspace, workspace_bytes, 0u,
+                           status, stream);
+}
+
+int32_t moe_expert_ffn_ex(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
+                          const int32_t* kept_cnt, void* H, void* ye, void* workspace,
+                          size_t workspace_bytes, uint32_t flags, int32_t* status,
+                          moe_stream_t stream) {
   set_last_error("");
+  if (flags & ~static_cast<uint32_t>(MOE_FFN_WORKSPACE_ZEROED))
+    return fail(MOE_ERR_INVALID_ARGUMENT, "moe_expert_ffn_ex: unknown flag bits");
   MOE_TRY(check_cfg(cfg));
   if (cfg->capacity == 0) return MOE_OK;
   MOE_TRY(need_ptr(xe, "xe"));
@@ -267,7 +287,8 @@ int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, co
     if (!workspace || workspace_bytes < need)
       return fail(MOE_ERR_WORKSPACE, "moe_expert_ffn: workspace needs " + std::to_string(need) + " bytes");
     MOE_TRY(need_ptr(workspace, "workspace"));
-    return launch_ffn_tc(*cfg, xe, W1, W2, kept_cnt, H, ye, workspace, false, status, s);
+    return launch_ffn_tc(*cfg, xe, W1, W2, kept_cnt, H, ye, workspace,
+                         (flags & MOE_FFN_WORKSPACE_ZEROED) != 0, status, s);
   }
   return launch_ffn_f32(*cfg, xe, W1, W2, kept_cnt, H, ye, s);
 }

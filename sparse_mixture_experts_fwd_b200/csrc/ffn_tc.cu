@@ -55,7 +55,8 @@ struct FfnParams {
   __nv_bfloat16* ye;
   unsigned int* tile_ctr;  // zero before launch
   unsigned int* done1;     // [E], zero before launch
-  int32_t* status;
+  int32_t* status;         // nullable; also the call's give-up signal
+  uint64_t wait_ns;        // limit of every bounded wait
   // top-1 layers: GEMM 2 writes gate * row straight to y [T, d] in token order
   // (ye untouched); null -> write ye
   const int32_t* tok_of_row;
@@ -114,18 +115,19 @@ MOE_DEV void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Bounded wait until *p >= need (acquire).  False on timeout / abort.
-MOE_DEV bool wait_count(const unsigned int* p, unsigned int need, volatile int* abort,
-                        int32_t* status) {
-  if (ld_acquire_u32(p) >= need) return true;
+// Bounded wait until *p has reached `need` (acquire), compared as the signed
+// difference *p - need >= 0, so a counter started below zero (a caller-set
+// state that no tile can complete) waits until the limit.  False on timeout /
+// give-up.
+MOE_DEV bool wait_count(const unsigned int* p, unsigned int need, const dev::Abort& ab) {
+  if (static_cast<int>(ld_acquire_u32(p) - need) >= 0) return true;
   const unsigned long long t0 = dev::globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (ld_acquire_u32(p) >= need) return true;
+    if (static_cast<int>(ld_acquire_u32(p) - need) >= 0) return true;
     if ((it & 15u) == 0) {
-      if (*abort) return false;
-      if (dev::globaltimer() - t0 > dev::kWaitLimitNs) {
-        *abort = 1;
-        if (status) atomicOr(status, MOE_STATUS_TIMEOUT);
+      if (ab.raised()) return false;
+      if (dev::globaltimer() - t0 > ab.limit_ns) {
+        ab.raise();
         return false;
       }
       __nanosleep(64);
@@ -185,11 +187,11 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     dev::tma_prefetch_desc(&tmH);
     dev::tma_prefetch_desc(&tmW2);
   }
-  if (warp == 1) {
+  dev::pdl_wait();  // kept counts, xe and the zeroed counters are visible from here
+  if (warp == 1) {  // TMEM only after the previous kernel has finished (see pdl_wait)
     dev::tmem_alloc(&s_tmem_base, kTmemCols);
     dev::tmem_relinquish();
   }
-  dev::pdl_wait();  // kept counts, xe and the zeroed counters are visible from here
   for (int e = tid; e < E; e += kThreads) {
     int r = p.kept_cnt[e];
     r = r < 0 ? 0 : (r > p.C ? p.C : r);
@@ -210,7 +212,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
   dev::tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
   const int total = s_prefix[sc.units];
-  volatile int* abort_flag = &s_abort;
+  const dev::Abort ab{&s_abort, p.status, p.wait_ns};
 
   if (warp == 0) {
     // ---------------- tile grabber + TMA producer ----------------
@@ -222,10 +224,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      while (!*abort_flag) {
+      while (!ab.raised()) {
         int t = static_cast<int>(atomicAdd(p.tile_ctr, 1u));
-        if (t >= total) t = -1;
-        if (!dev::mbar_wait(&ring_empty[slot], rphase ^ 1u, abort_flag, p.status)) break;
+        if (t < 0 || t >= total) t = -1;  // (negative only from a counter not zeroed)
+        if (!dev::mbar_wait(&ring_empty[slot], rphase ^ 1u, ab)) break;
         s_ring[slot] = t;
         dev::mbar_arrive(&ring_full[slot]);
         if (++slot == kRing) { slot = 0; rphase ^= 1u; }
@@ -238,14 +240,14 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         if (x.kind == 2) {
           // all GEMM-1 tiles of this expert must have stored H (4 warp arrivals per tile)
           const unsigned int need = static_cast<unsigned int>(4 * s_mblk[x.e] * sc.nb1);
-          if (!wait_count(p.done1 + x.e, need, abort_flag, p.status)) break;
+          if (!wait_count(p.done1 + x.e, need, ab)) break;
           fence_proxy_async_global();  // generic-proxy H stores -> async-proxy (TMA) reads
         }
         const int a_row = x.e * p.C + x.m * kBM;
         const int b_row = x.e * b_rows + x.n * kBN;
         bool ok = true;
         for (int kb = 0; kb < K / kBK; ++kb) {
-          if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, ab)) { ok = false; break; }
           dev::mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
           dev::tma_load_2d(smA + stage * kABytes, ta, &full_bar[stage], kb * kBK, a_row, pol_a);
           dev::tma_load_2d(smB + stage * kBBytes, tb, &full_bar[stage], kb * kBK, b_row, pol_w);
@@ -254,11 +256,11 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
         if (!ok) break;
       }
+      const unsigned long long deadline = dev::globaltimer() + p.wait_ns;
       for (int s = 0; s < kStages; ++s) {
         if (issued > s) {
           const long long last_fill = (issued - 1 - s) / kStages;
-          dev::mbar_wait(&full_bar[s], static_cast<uint32_t>(last_fill & 1), nullptr, p.status,
-                         abort_flag);
+          dev::mbar_wait_drain(&full_bar[s], static_cast<uint32_t>(last_fill & 1), ab, deadline);
         }
       }
     }
@@ -273,19 +275,19 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       uint32_t acc_phase = 0;
       bool any = false;
       while (true) {
-        if (!dev::mbar_wait(&ring_full[slot], rphase, abort_flag, p.status)) break;
+        if (!dev::mbar_wait(&ring_full[slot], rphase, ab)) break;
         const int t = s_ring[slot];
         dev::mbar_arrive(&ring_empty[slot]);
         if (++slot == kRing) { slot = 0; rphase ^= 1u; }
         if (t < 0) break;
         const Tile x = sc.decode(t);
         const int num_kb = (x.kind == 1 ? p.d : p.f) / kBK;
-        if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+        if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, ab)) break;
         dev::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!dev::mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          if (!dev::mbar_wait(&full_bar[stage], phase, ab)) { ok = false; break; }
           dev::tc_fence_after();
           const uint64_t adesc = dev::smem_desc_k_sw128(dev::smem_u32(smA + stage * kABytes));
           const uint64_t bdesc = dev::smem_desc_k_sw128(dev::smem_u32(smB + stage * kBBytes));
@@ -303,7 +305,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       }
       if (any) {
         dev::umma_commit(&done_bar);
-        dev::mbar_wait(&done_bar, 0, nullptr, p.status, abort_flag);
+        dev::mbar_wait_drain(&done_bar, 0, ab, dev::globaltimer() + p.wait_ns);
       }
     }
   } else {
@@ -317,7 +319,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     while (true) {
       int t = -1, ok = 0;
       if (lane == 0) {
-        ok = dev::mbar_wait(&ring_full[slot], rphase, abort_flag, p.status) ? 1 : 0;
+        ok = dev::mbar_wait(&ring_full[slot], rphase, ab) ? 1 : 0;
         if (ok) {
           t = s_ring[slot];
           dev::mbar_arrive(&ring_empty[slot]);
@@ -328,7 +330,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       if (!ok || t < 0) break;
       if (++slot == kRing) { slot = 0; rphase ^= 1u; }
       const Tile x = sc.decode(t);
-      if (lane == 0) ok = dev::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status) ? 1 : 0;
+      if (lane == 0) ok = dev::mbar_wait(&tfull_bar[acc], acc_phase, ab) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       dev::tc_fence_after();
@@ -435,8 +437,10 @@ int32_t make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 
 }  // namespace
 
+// tile counter, then one counter per (expert, chunk of at most 256 rows)
 size_t ffn_sync_bytes(const moe_config& c) {
-  return align256(sizeof(unsigned int) * (1 + static_cast<size_t>(c.E)));
+  return align256(sizeof(unsigned int) *
+                  (1 + static_cast<size_t>(c.E) * static_cast<size_t>(ffn_pair_chunks(c))));
 }
 
 int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const void* W2,
@@ -445,10 +449,11 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
   if (C >= 512) {
-    // Experts with hundreds of rows make the GEMMs tensor-core bound; SM
-    // pairs (256 x 256 tiles, cta_group::2) feed each SM a third fewer operand
-    // bytes per flop than single-CTA 128 x 256 tiles.
-    return launch_ffn_pairs(c, xe, W1, W2, kept_cnt, H, ye, status, s, top1);
+    // Experts with hundreds of rows make the GEMMs tensor-core bound: both
+    // GEMMs on SM pairs in one launch, tokens in 16-row steps on the MMA's N
+    // side so a ragged expert wastes almost no MMA rows.
+    return launch_ffn_pair_fused(c, xe, W1, W2, kept_cnt, H, ye, sync, sync_zeroed, status, s,
+                                 top1);
   }
   if (C > kBM) {
     // Experts span several 128-row blocks: several CTAs share each weight
@@ -490,6 +495,7 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
   p.tile_ctr = static_cast<unsigned int*>(sync);
   p.done1 = static_cast<unsigned int*>(sync) + 1;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   if (top1) {
     p.tok_of_row = top1->tok_of_row;
     p.gate = top1->gate;

@@ -58,7 +58,8 @@ struct GemmParams {
   const int32_t* scatter_tok;  // EPI_BF16, top-1 layers: row -> token map, or null
   const float* scatter_gate;   //   gate per token
   __nv_bfloat16* scatter_y;    //   y [T, out_ld] written instead of out
-  int32_t* status;             // nullable
+  int32_t* status;             // nullable; also the call's give-up signal
+  uint64_t wait_ns;            // limit of every bounded wait
 };
 
 template <int BN>
@@ -141,11 +142,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     dev::tma_prefetch_desc(&tmA);
     dev::tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) {
+  dev::pdl_wait();  // the previous kernel's outputs (row counts, x) are visible from here
+  if (warp == 1) {  // TMEM only after the previous kernel has finished (see pdl_wait)
     dev::tmem_alloc(&s_tmem_base, C::kTmemCols);
     dev::tmem_relinquish();
   }
-  dev::pdl_wait();  // the previous kernel's outputs (row counts, x) are visible from here
   for (int g = tid; g < G; g += kThreads) {
     int r = p.group_rows ? p.group_rows[g] : p.fixed_rows;
     r = r < 0 ? 0 : (r > p.max_rows ? p.max_rows : r);
@@ -170,7 +171,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   dev::tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
   const int total_tiles = s_prefix[G];
-  volatile int* abort_flag = &s_abort;
+  const dev::Abort ab{&s_abort, p.status, p.wait_ns};
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -178,12 +179,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+      for (int t = blockIdx.x; t < total_tiles && !ab.raised(); t += gridDim.x) {
         TileCoord tc = tile_of(t, s_prefix, s_mblk, G, n_blocks);
         const int a_row = tc.g * p.a_group_rows + tc.m_blk * kBM;
         const int b_row = tc.g * p.b_group_rows + tc.n_blk * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) break;
+          if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, ab)) break;
           dev::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
           dev::tma_load_2d(smA + stage * C::kABytes, &tmA, &full_bar[stage], kb * kBK, a_row);
           dev::tma_load_2d(smB + stage * C::kBBytes, &tmB, &full_bar[stage], kb * kBK, b_row);
@@ -192,11 +193,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       }
       // Make sure no bulk copy is still landing in shared memory when the CTA exits.
+      const unsigned long long deadline = dev::globaltimer() + p.wait_ns;
       for (int s = 0; s < S; ++s) {
         if (issued > s) {
           long long last_fill = (issued - 1 - s) / S;
-          dev::mbar_wait(&full_bar[s], static_cast<uint32_t>(last_fill & 1), nullptr, p.status,
-                         abort_flag);
+          dev::mbar_wait_drain(&full_bar[s], static_cast<uint32_t>(last_fill & 1), ab, deadline);
         }
       }
     }
@@ -208,13 +209,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
-      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
-        if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+      for (int t = blockIdx.x; t < total_tiles && !ab.raised(); t += gridDim.x) {
+        if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, ab)) break;
         dev::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!dev::mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          if (!dev::mbar_wait(&full_bar[stage], phase, ab)) { ok = false; break; }
           dev::tc_fence_after();
           const uint64_t adesc = dev::smem_desc_k_sw128(dev::smem_u32(smA + stage * C::kABytes));
           const uint64_t bdesc = dev::smem_desc_k_sw128(dev::smem_u32(smB + stage * C::kBBytes));
@@ -235,7 +236,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (any) {
         // every MMA issued by this thread has completed before TMEM is released
         dev::umma_commit(&done_bar);
-        dev::mbar_wait(&done_bar, 0, nullptr, p.status, abort_flag);
+        dev::mbar_wait_drain(&done_bar, 0, ab, dev::globaltimer() + p.wait_ns);
       }
     }
   } else {
@@ -249,7 +250,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // lane 0 waits; the result is broadcast so the warp stays converged for
       // the .sync.aligned tcgen05.ld below
       int ok = 0;
-      if (lane == 0) ok = dev::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status) ? 1 : 0;
+      if (lane == 0) ok = dev::mbar_wait(&tfull_bar[acc], acc_phase, ab) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       dev::tc_fence_after();
@@ -486,6 +487,7 @@ int32_t launch_ffn_two_pass(const moe_config& c, const void* xe, const void* W1,
   p.fixed_rows = 0;
   p.max_rows = c.capacity;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   p.bias = nullptr;
   // GEMM 1: [E*C, d] x [E*f, d]^T -> H [E*C, f], ReLU; GEGLU: W1 has 2f rows
   // per expert and each pair of accumulator columns gives one unit of H
@@ -531,6 +533,7 @@ int32_t launch_router_tc(const moe_config& c, const void* x, const void* Wr, con
   p.out_ld = c.E;
   p.bias = bias;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   const int64_t tiles = (c.T + kBM - 1) / kBM;
   const uint64_t T = static_cast<uint64_t>(c.T), E = static_cast<uint64_t>(c.E);
   if (c.E <= 32) return launch_gemm<32, EPI_F32_BIAS>(x, T, Wr, E, p, tiles, s);
@@ -564,6 +567,7 @@ int32_t launch_router_topk_tc(const moe_config& c, const void* x, const void* Wr
   p.clear = clear;
   p.n_clear = n_clear;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   const int64_t tiles = (c.T + kBM - 1) / kBM;
   const uint64_t T = static_cast<uint64_t>(c.T), E = static_cast<uint64_t>(c.E);
   if (c.E <= 32) return launch_gemm<32, EPI_TOPK>(x, T, Wr, E, p, tiles, s);

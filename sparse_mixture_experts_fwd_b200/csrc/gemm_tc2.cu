@@ -56,7 +56,8 @@ struct Gemm2Params {
   int32_t K;
   __nv_bfloat16* out;
   int64_t out_ld;
-  int32_t* status;
+  int32_t* status;             // nullable; also the call's give-up signal
+  uint64_t wait_ns;            // limit of every bounded wait
   const int32_t* scatter_tok;  // EPI2_BF16, top-1 layers: row -> token map, or null
   const float* scatter_gate;   //   gate per token
   __nv_bfloat16* scatter_y;    //   y [T, out_ld] written instead of out
@@ -184,11 +185,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     dev::tma_prefetch_desc(&tmA);
     dev::tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) {
+  dev::pdl_wait();
+  if (warp == 1) {  // TMEM only after the previous kernel has finished (see pdl_wait)
     tmem_alloc2(&s_tmem_base, kTmemCols);
     tmem_relinquish2();
   }
-  dev::pdl_wait();
   for (int g = tid; g < G; g += kThreads) {
     int r = p.group_rows[g];
     r = r < 0 ? 0 : (r > p.max_rows ? p.max_rows : r);
@@ -210,7 +211,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   dev::tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
   const int total = s_prefix[G];
-  volatile int* abort_flag = &s_abort;
+  const dev::Abort ab{&s_abort, p.status, p.wait_ns};
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -218,12 +219,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = cluster; t < total && !*abort_flag; t += n_clusters) {
+      for (int t = cluster; t < total && !ab.raised(); t += n_clusters) {
         const TileCoord tc = tile_of(t, s_prefix, s_mblk, G);
         const int a_row = tc.g * p.a_group_rows + tc.m * kBM + static_cast<int>(rank) * kHalf;
         const int b_row = tc.g * p.b_group_rows + tc.n * kBN + static_cast<int>(rank) * kHalf;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.status)) break;
+          if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, ab)) break;
           if (rank == 0) dev::mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
           const uint32_t full0 = mapa(&full_bar[stage], 0);  // CTA 0's barrier for this stage
           tma_load_2d_pair(smA + stage * kABytes, &tmA, full0, kb * kBK, a_row);
@@ -234,11 +235,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       }
       if (rank == 0) {
         // the pair's copies have all landed once CTA 0's full barriers complete
+        const unsigned long long deadline = dev::globaltimer() + p.wait_ns;
         for (int s = 0; s < kStages; ++s) {
           if (issued > s) {
             const long long last_fill = (issued - 1 - s) / kStages;
-            dev::mbar_wait(&full_bar[s], static_cast<uint32_t>(last_fill & 1), nullptr, p.status,
-                           abort_flag);
+            dev::mbar_wait_drain(&full_bar[s], static_cast<uint32_t>(last_fill & 1), ab, deadline);
           }
         }
       }
@@ -251,13 +252,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
-      for (int t = cluster; t < total && !*abort_flag; t += n_clusters) {
-        if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+      for (int t = cluster; t < total && !ab.raised(); t += n_clusters) {
+        if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, ab)) break;
         dev::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!dev::mbar_wait(&full_bar[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          if (!dev::mbar_wait(&full_bar[stage], phase, ab)) { ok = false; break; }
           dev::tc_fence_after();
           const uint64_t adesc = dev::smem_desc_k_sw128(dev::smem_u32(smA + stage * kABytes));
           const uint64_t bdesc = dev::smem_desc_k_sw128(dev::smem_u32(smB + stage * kBBytes));
@@ -274,7 +275,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       }
       if (any) {
         umma2_commit_local(&done_bar);
-        dev::mbar_wait(&done_bar, 0, nullptr, p.status, abort_flag);
+        dev::mbar_wait_drain(&done_bar, 0, ab, dev::globaltimer() + p.wait_ns);
       }
     }
   } else {
@@ -288,7 +289,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     for (int t = cluster; t < total; t += n_clusters) {
       const TileCoord tc = tile_of(t, s_prefix, s_mblk, G);
       int ok = 0;
-      if (lane == 0) ok = dev::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, p.status) ? 1 : 0;
+      if (lane == 0) ok = dev::mbar_wait(&tfull_bar[acc], acc_phase, ab) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       dev::tc_fence_after();
@@ -433,6 +434,7 @@ int32_t launch_ffn_pairs(const moe_config& c, const void* xe, const void* W1, co
   p.group_rows = kept_cnt;
   p.max_rows = c.capacity;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   // GEGLU: W1 has 2f rows per expert, each accumulator column pair one unit of H
   const bool glu = c.expert == MOE_EXPERT_GEGLU;
   const int64_t n1 = glu ? 2 * f : f;

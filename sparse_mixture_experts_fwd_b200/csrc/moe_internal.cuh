@@ -21,6 +21,7 @@ const char* last_error_cstr();
 int32_t fail(int32_t code, const std::string& msg);
 int32_t check_launch(const char* what);  // maps cudaGetLastError to MOE_ERR_CUDA
 int num_sms();                            // SM count of the current device (cached)
+uint64_t wait_limit_ns();                 // limit of every bounded wait, for the next launches
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -68,6 +69,13 @@ size_t ffn_sync_bytes(const moe_config& c);
 int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const void* W2,
                       const int32_t* kept_cnt, void* H, void* ye, void* sync, bool sync_zeroed,
                       int32_t* status, cudaStream_t s, const Top1Out* top1 = nullptr);
+// C >= 512: both GEMMs in one persistent launch on SM pairs; sync as above
+// (ffn_sync_bytes), chunks of at most 256 rows per expert
+int ffn_pair_chunks(const moe_config& c);
+int32_t launch_ffn_pair_fused(const moe_config& c, const void* xe, const void* W1, const void* W2,
+                              const int32_t* kept_cnt, void* H, void* ye, void* sync,
+                              bool sync_zeroed, int32_t* status, cudaStream_t s,
+                              const Top1Out* top1 = nullptr);
 int32_t launch_ffn_f32(const moe_config& c, const void* xe, const void* W1, const void* W2,
                        const int32_t* kept_cnt, void* H, void* ye, cudaStream_t s);
 int32_t launch_route_assign(const moe_config& c, const float* logits, const int32_t* domain,
@@ -119,14 +127,37 @@ int32_t launch_ep_combine(const moe_config& c, int rank, int world, const void* 
 namespace moe {
 namespace dev {
 
-// Wall-clock limit of every spin-wait in the library's kernels.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+// Wall-clock limit of every spin-wait in the library's kernels, unless the
+// host sets another with moe_set_wait_limit_ns (kernels take it as a parameter).
+constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;  // 1 s
 
 MOE_DEV unsigned long long globaltimer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+// The give-up signal that all bounded waits of a kernel share.  `status` is
+// the call's status word: its MOE_STATUS_TIMEOUT bit, once any CTA of any
+// kernel of the call sets it, makes every other wait of the call give up at
+// its next poll, so one expired wait ends the whole grid (and the kernels
+// after it on the stream) within about one poll interval instead of each
+// CTA spending its own limit.  `local` is the CTA's own flag, the only
+// signal when the caller passed no status word.
+struct Abort {
+  volatile int* local;
+  int32_t* status;
+  unsigned long long limit_ns;
+
+  MOE_DEV bool raised() const {
+    if (*local) return true;
+    return status && (*reinterpret_cast<volatile int32_t*>(status) & MOE_STATUS_TIMEOUT);
+  }
+  MOE_DEV void raise() const {
+    *local = 1;
+    if (status) atomicOr(status, MOE_STATUS_TIMEOUT);
+  }
+};
 
 MOE_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -138,7 +169,11 @@ MOE_DEV uint32_t lane_id() { return threadIdx.x & 31u; }
 // with programmatic stream serialisation: it lets the next kernel start
 // early (pdl_trigger at entry) and performs pdl_wait, which returns once the
 // previous kernel on the stream has completed and its writes are visible,
-// before its first global-memory read or write.
+// before its first global-memory read or write.  Tensor memory is allocated
+// only after pdl_wait: a CTA that took TMEM before it and landed on an SM
+// whose CTA of the previous kernel had triggered but not yet allocated
+// would block that allocation (tcgen05.alloc waits for free columns) while
+// itself waiting for that kernel to finish.
 MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -167,24 +202,34 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase of `parity` to complete, for at most kWaitLimitNs, or
-// until *abort becomes non-zero (abort nullable: then only the time limit
-// applies).  Returns false on timeout/abort; a timeout sets *abort and ORs
-// MOE_STATUS_TIMEOUT into *status (nullable).
-MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status,
-                       volatile int* abort_to_set = nullptr) {
+// Wait for the phase of `parity` to complete, for at most ab.limit_ns, or
+// until the give-up signal is raised.  False on timeout / give-up; a timeout
+// raises the signal (sets the CTA flag and the status word's timeout bit).
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (abort && *abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        if (abort) *abort = 1;
-        if (abort_to_set) *abort_to_set = 1;
-        if (status) atomicOr(status, MOE_STATUS_TIMEOUT);
+      if (ab.raised()) return false;
+      if (globaltimer() - t0 > ab.limit_ns) {
+        ab.raise();
         return false;
       }
+    }
+  }
+}
+// The waits a CTA makes before it exits, for copies and MMAs it has already
+// issued: they ignore the give-up signal (the hardware is still writing this
+// CTA's shared memory or tensor memory) and share one absolute deadline, so
+// the whole drain takes at most one limit.
+MOE_DEV bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const Abort& ab,
+                             unsigned long long deadline) {
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 63u && globaltimer() > deadline) {
+      ab.raise();
+      return false;
     }
   }
 }

@@ -176,22 +176,27 @@ struct AssignArgs {
   unsigned int* flags;  // [nblk], cleared before launch
   int32_t* aggr;        // [nblk][E]
   int32_t* incl;        // [nblk][E]
-  int32_t* status;
+  int32_t* status;      // nullable; also the call's give-up signal
+  uint64_t wait_ns;     // limit of the look-back wait
 };
 
 __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArgs p) {
   extern __shared__ int s_cnt[];  // [32 warps][E], then excl[E]
-  __shared__ int s_pstar, s_ok, s_maxinc, s_maxbad, s_drop[32];
+  __shared__ int s_pstar, s_ok, s_maxinc, s_maxbad, s_drop[32], s_ticket;
   int* s_excl = s_cnt + 32 * p.E;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.x;
   const int E = p.E;
 
   // 1. ranks inside the block
   dev::pdl_trigger();
   for (int i = tid; i < 32 * E; i += kAssignBlock) s_cnt[i] = 0;
   dev::pdl_wait();
+  // The block's place in token order is a ticket taken when it starts, not
+  // blockIdx: a block then only ever waits on blocks that are already running,
+  // whatever order the hardware starts them in.
+  if (tid == 0) s_ticket = static_cast<int>(atomicAdd(p.flags + p.nblk, 1u));
   __syncthreads();
+  const int b = s_ticket;
   const int64_t a = static_cast<int64_t>(b) * kAssignBlock + tid;
   int e = a < p.n_assign ? __ldg(p.expert_idx + a) : -1;
   if (e >= E) e = -1;
@@ -235,8 +240,17 @@ __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArg
       const bool ready = s_maxinc >= 0 && s_maxbad < s_maxinc;
       if (tid == 0) {
         s_pstar = s_maxinc;
-        s_ok = ready ? 1 : (dev::globaltimer() - t0 > dev::kWaitLimitNs ? -1 : 0);
-        if (s_ok < 0 && p.status) atomicOr(p.status, MOE_STATUS_TIMEOUT);
+        if (ready) {
+          s_ok = 1;
+        } else if (p.status &&
+                   (*reinterpret_cast<volatile int32_t*>(p.status) & MOE_STATUS_TIMEOUT)) {
+          s_ok = -1;  // another wait of this call has already given up
+        } else if (dev::globaltimer() - t0 > p.wait_ns) {
+          s_ok = -1;
+          if (p.status) atomicOr(p.status, MOE_STATUS_TIMEOUT);
+        } else {
+          s_ok = 0;
+        }
       }
       __syncthreads();
       if (s_ok != 0) break;
@@ -324,14 +338,15 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace
 
+// the look-back flags [nblk] and the block ticket counter after them
 int assign_flag_words(const moe_config& c) {
-  return static_cast<int>(ceil_div(c.T * c.k, kAssignBlock));
+  return static_cast<int>(ceil_div(c.T * c.k, kAssignBlock)) + 1;
 }
 
-// flags [nblk] u32, then aggr and incl [nblk][E] i32 each
+// flags [nblk] u32 + ticket u32, then aggr and incl [nblk][E] i32 each
 size_t assign_scratch_bytes(const moe_config& c) {
   const int64_t nblk = ceil_div(c.T * c.k, kAssignBlock);
-  return align256(static_cast<size_t>(nblk) * sizeof(unsigned int)) +
+  return align256(static_cast<size_t>(nblk + 1) * sizeof(unsigned int)) +
          2 * align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
 }
 
@@ -354,7 +369,7 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
   const int64_t nblk = ceil_div(n_assign, kAssignBlock);
   char* sc = static_cast<char*>(scratch);
   unsigned int* flags = reinterpret_cast<unsigned int*>(sc);
-  const size_t flags_bytes = align256(static_cast<size_t>(nblk) * sizeof(unsigned int));
+  const size_t flags_bytes = align256(static_cast<size_t>(nblk + 1) * sizeof(unsigned int));
   const size_t vec_bytes = align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
   int32_t* aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
   int32_t* incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
@@ -367,16 +382,16 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
     const int64_t blocks = std::min<int64_t>(ceil_div(T, 8), int64_t(num_sms()) * 16);
     if (c.k == 1)
       launch_pdl(gate_topk_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
-                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
+                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk + 1));
     else
       launch_pdl(gate_topk_kernel<2>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
-                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk));
+                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk + 1));
     int32_t rc = check_launch("gate_topk_kernel");
     if (rc != MOE_OK) return rc;
   } else {
     launch_pdl(route_rre_kernel, dim3(static_cast<unsigned>(ceil_div(T, 256))), dim3(256), 0, s,
                T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status, flags,
-               static_cast<int>(nblk));
+               static_cast<int>(nblk + 1));
     int32_t rc = check_launch("route_rre_kernel");
     if (rc != MOE_OK) return rc;
   }
@@ -397,7 +412,7 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
     return check_launch("assign_empty_kernel");
   }
   char* sc = static_cast<char*>(scratch);
-  const size_t flags_bytes = align256(static_cast<size_t>(nblk) * sizeof(unsigned int));
+  const size_t flags_bytes = align256(static_cast<size_t>(nblk + 1) * sizeof(unsigned int));
   const size_t vec_bytes = align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
   AssignArgs p{};
   p.n_assign = n_assign;
@@ -416,6 +431,7 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
   p.aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
   p.incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
   p.status = status;
+  p.wait_ns = wait_limit_ns();
   const size_t smem = (33 * static_cast<size_t>(c.E)) * sizeof(int);
   launch_pdl(assign_kernel, dim3(static_cast<unsigned>(nblk)), dim3(kAssignBlock), smem, s, p);
   return check_launch("assign_kernel");

@@ -14,6 +14,7 @@
 // (kSegsPerLaunch per launch), so no host->device copy is needed.
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 #include "moe_internal.cuh"
@@ -266,8 +267,6 @@ extern "C" int32_t sparseclip_clip(float* const* dense, const int64_t* dense_len
 // other host threads) race and must be serialised by the caller.
 // ---------------------------------------------------------------------------
 
-#include <mutex>
-
 namespace moe {
 namespace {
 
@@ -277,24 +276,54 @@ constexpr int kStaticMaxLaunches = kStaticMaxSegs / kSegsPerLaunch;
 static __device__ __align__(256) double g_static_partials[kStaticMaxLaunches * kGrid * 2];
 
 std::mutex g_static_mu;
-double* g_static_ptr[64] = {};
+// The array's address belongs to one CUDA context: it is looked up with the
+// device current and cached per (device, context), so a caller that switches
+// to another context on the device (or resets the device) gets a fresh lookup.
+struct StaticAddr {
+  CUcontext ctx;
+  double* ptr;
+};
+StaticAddr g_static_addr[64] = {};
 
-// Device address of g_static_partials on the current device, looked up once
-// per device (with that device current) on the first call made there.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  return fn;
+}
+
+// Device address of g_static_partials in the current context, looked up with
+// cudaGetSymbolAddress on the first call made with each device / context
+// current (so that first call should come before any stream capture).
 int32_t static_partials(double** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
   if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal >= 64");
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (!get) return fail(MOE_ERR_CUDA, "cuCtxGetCurrent unavailable from the driver");
+  CUcontext ctx = nullptr;  // null before the runtime has made a context current
+  if (get(&ctx) != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuCtxGetCurrent failed");
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  StaticAddr& a = g_static_addr[dev];
+  if (!ctx || !a.ptr || a.ctx != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_partials);
+    e = cudaGetSymbolAddress(&p, g_static_partials);  // makes the device's context current
     if (e != cudaSuccess || !p)
       return fail(MOE_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-    g_static_ptr[dev] = static_cast<double*>(p);
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return fail(MOE_ERR_CUDA, "cuCtxGetCurrent failed");
+    a.ctx = ctx;
+    a.ptr = static_cast<double*>(p);
   }
-  *out = g_static_ptr[dev];
+  *out = a.ptr;
   return MOE_OK;
 }
 

@@ -15,6 +15,12 @@ need from ``torch.distributed``:
   (a one-word all-reduce; on NCCL it is ordered on the current stream, so
   the host never waits).
 
+``sync="host"`` orders the steps from the host instead, for process groups
+whose backend cannot order work on a CUDA stream (gloo): each barrier is a
+``torch.cuda.synchronize()`` followed by a group barrier, and the kept counts
+travel as CPU tensors.  No kernel then ever waits for another process, which
+also lets several ranks share one GPU.
+
 Each rank's output equals the single-device layer on that rank's batch: the
 capacity C applies per batch and expert e's buffer on its home rank holds the
 world * C rows its senders may keep.
@@ -28,18 +34,36 @@ from . import (ROUTE_TOPK, _act_dtype, assign_workspace_size, ep_combine,
                ep_dispatch, ep_ffn_config, expert_ffn, ffn_workspace_size, router, topk_assign)
 
 
-def exchange_counts(kept_cnt: torch.Tensor, world: int, group=None, out=None) -> torch.Tensor:
-    """cnt_all [world, E]: row q = rank q's kept counts (an all-gather)."""
+def exchange_counts(kept_cnt: torch.Tensor, world: int, group=None, out=None,
+                    host: bool = False) -> torch.Tensor:
+    """cnt_all [world, E]: row q = rank q's kept counts (an all-gather).
+
+    ``host``: gather CPU copies (after the counts are final) and copy the
+    result into ``out`` (or a new tensor on the counts' device)."""
     E = kept_cnt.numel()
+    if host:
+        parts = [torch.empty(E, dtype=torch.int32) for _ in range(world)]
+        dist.all_gather(parts, kept_cnt.detach().to("cpu", torch.int32).view(-1), group=group)
+        full = torch.stack(parts)
+        if out is None:
+            return full.to(kept_cnt.device)
+        out.view(world, E).copy_(full)
+        return out.view(world, E)
     flat = out.view(-1) if out is not None else torch.empty(world * E, dtype=torch.int32,
                                                             device=kept_cnt.device)
     dist.all_gather_into_tensor(flat, kept_cnt.contiguous().view(-1), group=group)
     return flat.view(world, E)
 
 
-def rank_barrier(token: torch.Tensor, group=None) -> None:
+def rank_barrier(token: torch.Tensor, group=None, host: bool = False) -> None:
     """Every rank's work enqueued before this call completes before any
-    rank's work enqueued after it (``token``: a zero word, kept zero)."""
+    rank's work enqueued after it (``token``: a zero word, kept zero).
+    ``host``: wait for this process's GPU work, then meet the other ranks."""
+    if host:
+        if torch.cuda.is_initialized():  # a process that never used CUDA has nothing to wait for
+            torch.cuda.synchronize()
+        dist.barrier(group=group)
+        return
     dist.all_reduce(token, group=group)
 
 
@@ -71,7 +95,10 @@ class ExpertParallelLayer:
     rank's T and capacity C); ``forward`` takes this rank's expert shards
     W1 [E/world, f (2f for GEGLU), d] and W2 [E/world, d, f]."""
 
-    def __init__(self, cfg, group=None, device=None):
+    def __init__(self, cfg, group=None, device=None, sync: str = "stream"):
+        if sync not in ("stream", "host"):
+            raise ValueError('sync must be "stream" or "host"')
+        self.host_sync = sync == "host"
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
@@ -114,13 +141,14 @@ class ExpertParallelLayer:
             router(cfg, x, Wr, bias, logits=self.logits, status=status)
         r = topk_assign(cfg, logits=self.logits, domain_id=domain_id, out=self.route,
                         workspace=self.assign_ws, status=status)
-        exchange_counts(r["kept_cnt"], world, g, out=self.cnt_all)
+        hs = self.host_sync
+        exchange_counts(r["kept_cnt"], world, g, out=self.cnt_all, host=hs)
         ep_dispatch(cfg, rank, world, x, r["expert_idx"], r["slot"], r["kept"], self.cnt_all,
                     self.xe_peers, local_cnt=self.local_cnt, status=status)
-        rank_barrier(self.token, g)  # every rank's rows have landed
+        rank_barrier(self.token, g, host=hs)  # every rank's rows have landed
         expert_ffn(self.ffn_cfg, self.xe, W1_local, W2_local, self.local_cnt, H=self.H, ye=self.ye,
                    workspace=self.ffn_ws, status=status)
-        rank_barrier(self.token, g)  # every rank's expert outputs are written
+        rank_barrier(self.token, g, host=hs)  # every rank's expert outputs are written
         y = ep_combine(cfg, rank, world, self.ye_peers, r["expert_idx"], r["gate"], r["slot"],
                        r["kept"], self.cnt_all, y=y, status=status)
         return y

@@ -202,7 +202,7 @@ def test_library_refuses_cpu_tensors(moe):
 
 
 def _expected_check(T, d, f, E, k, C, mode, G, dtype, expert):
-    """The documented validity rules of moe_config, restated (header and DESIGN)."""
+    """The validity rules of moe_config as the C header documents them, restated."""
     I32 = 2 ** 31 - 1
     if T < 0 or T > I32 or E < 1:
         return -1

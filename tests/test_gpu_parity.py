@@ -203,6 +203,9 @@ FFN_SHAPES = {
     "sm_pairs_long_k": (3, 600, 512, 2048, [600, 0, 513]),
     # C > 512: last 256-row blocks holding 188, 100 (the only block), 128 and 89 rows
     "sm_pairs_tails": (5, 700, 256, 512, [700, 100, 0, 640, 601]),
+    # C >= 512, token chunks of every size class (1, 15, 16, 17 ... 513 rows), feature
+    # blocks cut short in both GEMMs (d = 192, f = 320)
+    "sm_pairs_chunks": (10, 600, 192, 320, [1, 15, 16, 17, 255, 256, 257, 511, 513, 600]),
     # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
     "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
 }
@@ -353,6 +356,51 @@ def test_layer_forward_full(moe, cuda_device, case):
             assert_close(v["ye"][e, s], yr, what=f"ye[{e},{s}]")
         assert torch.equal(v["xe"][e, s].view(torch.int16) if w.dtype == "bf16" else v["xe"][e, s],
                            inp["x"][t].view(torch.int16) if w.dtype == "bf16" else inp["x"][t])
+
+
+def test_layer_forward_whole_experts(moe, cuda_device, case):
+    """Every kept row of two whole experts at full size, element by element:
+    the most loaded expert (its last, ragged row block included) and one
+    drawn at random.  H and ye (or, for top-1 bf16 layers, whose combine runs
+    in the FFN, y of each row's token) against the oracle's expert network."""
+    w, inp, ref, D = case.w, case.inp, case.ref, case.dev
+    dev = cuda_device
+    C = case.C
+    cfg = case.cfg
+    ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    st = zero_status(dev)
+    y = moe.layer_forward(cfg, D["x"], D["W1"], D["W2"], Wr=D["Wr"], bias=D["bias"],
+                          domain_id=D["domain"], workspace=ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    views = moe.workspace_views(cfg, ws)
+    gidx = views["expert_idx"].cpu()
+    a = oracle.assign(gidx, w.E, C)  # the GPU's own choices (bit-exact slots checked elsewhere)
+    kept_cnt = a["kept_cnt"]
+    g = torch.Generator().manual_seed(11)
+    busiest = int(torch.argmax(kept_cnt))
+    others = [e for e in range(w.E) if e != busiest and int(kept_cnt[e]) > 0]
+    experts = [busiest] + ([others[int(torch.randint(0, len(others), (1,), generator=g))]]
+                           if others else [])
+    tok_of_row = a["tok_of_row"].view(w.E, C)
+    fused_top1 = w.k == 1 and w.dtype == "bf16"
+    y = y.cpu()
+    for e in experts:
+        n = int(kept_cnt[e])
+        toks = tok_of_row[e, :n].long()
+        xe = inp["x"][toks].unsqueeze(0).contiguous()
+        ye_ref, H_ref = oracle.expert_ffn(xe, inp["W1"][e:e + 1].contiguous(),
+                                          inp["W2"][e:e + 1].contiguous(),
+                                          torch.tensor([n], dtype=torch.int32), with_H=True,
+                                          nthreads=threads())
+        tol = dict(atol=1e-5, rtol=1e-5) if w.dtype == "f32" else {}
+        assert_close(views["H"][e, :n].cpu(), H_ref[0], what=f"H[{e}] ({n} rows)", **tol)
+        if not fused_top1:
+            assert_close(views["ye"][e, :n].cpu(), ye_ref[0], what=f"ye[{e}] ({n} rows)", **tol)
+        else:
+            # y[t] = gate_t * E(x_t), one rounding (the oracle rounds the expert output first)
+            gate = views["gate"].cpu()[toks, 0].double().unsqueeze(1)
+            assert_close(y[toks], gate * ye_ref[0].double(), what=f"y of expert {e}'s tokens")
 
 
 def test_layer_forward_deterministic(moe, cuda_device, case):

@@ -68,7 +68,12 @@ def _ep_worker(rank, world, port, q):
         cnt_all = exchange_counts(kept_cnt, world, out=out)
         token = torch.zeros(1, dtype=torch.int32)
         rank_barrier(token)
-        q.put((rank, cnt_all.data_ptr() == out.data_ptr(), cnt_all.tolist(), int(token.item())))
+        # the host-ordered form (gloo groups, ranks sharing a GPU): CPU all-gather
+        out_h = torch.full((world, E), -1, dtype=torch.int32)
+        cnt_h = exchange_counts(kept_cnt, world, out=out_h, host=True)
+        rank_barrier(token, host=True)
+        q.put((rank, cnt_all.data_ptr() == out.data_ptr(), cnt_all.tolist(), int(token.item()),
+               cnt_h.tolist(), cnt_h.data_ptr() == out_h.data_ptr()))
     finally:
         dist.destroy_process_group()
 
@@ -89,7 +94,7 @@ def test_expert_parallel_count_exchange_gloo():
         p.join(timeout=60)
         assert p.exitcode == 0
     want = [[(e * (r + 1)) % 7 for e in range(12)] for r in range(world)]
-    for rank, in_place, cnt_all, token in res:
-        assert in_place
-        assert cnt_all == want
+    for rank, in_place, cnt_all, token, cnt_h, in_place_h in res:
+        assert in_place and in_place_h
+        assert cnt_all == want and cnt_h == want
         assert token == 0

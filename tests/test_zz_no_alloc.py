@@ -5,7 +5,8 @@ start-up, or code that must not call the CUDA allocator where it runs).
 The entry point keeps its partial sums in a fixed array inside the library
 instead of a caller workspace.  This test calls it through the C ABI twice in
 a row, on different gradients, and checks each result against the
-workspace-taking sparseclip_norm on the same inputs.  It lives in its own file
+workspace-taking sparseclip_norm on the same inputs and against the CPU
+oracle's norm.  It lives in its own file
 that pytest collects last and passes alone in a fresh process as well as
 after the other tests.
 """
@@ -14,6 +15,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -59,6 +61,8 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
         torch.cuda.synchronize()
         got, want = out.cpu(), ref.cpu()
         assert bool(((got - want).abs() <= RTOL * want.abs()).all()), (got, want)
+        norm = oracle.sparseclip_norm([t.cpu() for t in dense], [t.cpu() for t in sparse], E)
+        assert abs(float(got[0]) - norm) <= RTOL * norm, (float(got[0]), norm)
 
 
 def test_noalloc_rejects_too_many_tensors(cuda_device):
