@@ -677,6 +677,9 @@ def run_b200(args, w, world, rank, local):
                        "(each record serialises the stream); frac = roofline time / stage time",
         "expert_ffn_tflops": ffn_flops / ffn_s / 1e12,
         "dispatch_combine_gbs": (disp_bytes + comb_bytes) / dc_s / 1e9,
+        "dispatch_combine_scope": ("dispatch only: the top-1 combine (the y scatter) runs inside "
+                                   "the expert FFN's GEMM-2 epilogue and is timed with expert_ffn"
+                                   if fused_combine else "dispatch and combine kernels"),
         "combine": "fused into the expert FFN's GEMM-2 epilogue" if fused_combine else "kernel",
         "aux_loss": aux,
         "sparseclip": sclip,

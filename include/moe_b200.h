@@ -53,7 +53,7 @@ extern "C" {
 
 typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 enum moe_error {
   MOE_OK = 0,
@@ -75,8 +75,11 @@ enum moe_expert { MOE_EXPERT_RELU = 0, MOE_EXPERT_GEGLU = 1 };
 enum moe_status_bits {
   MOE_STATUS_TIMEOUT = 1,   /* a pipeline wait gave up (wait limit); outputs invalid  */
   MOE_STATUS_BAD_DOMAIN = 2, /* an RRE domain id was outside 0..G-1 (routed as 0)      */
-  MOE_STATUS_BAD_COUNTS = 4  /* expert parallel: a row fell outside its expert's block
+  MOE_STATUS_BAD_COUNTS = 4, /* expert parallel: a row fell outside its expert's block
                                 (counts that do not match the assignment); skipped     */
+  MOE_STATUS_BAD_INDEX = 8   /* bounds-checked build only (moe_bounds_checked() == 1):
+                                moe_dispatch / moe_combine met an expert index outside
+                                0..E-1 or a slot outside 0..C-1; that choice skipped  */
 };
 
 /* One MoE layer.  56 bytes, no padding. */
@@ -128,6 +131,16 @@ size_t moe_workspace_map_size(void);
 const char* moe_error_string(int32_t code);
 /* Detail of the last error returned on the calling host thread ("" if none). */
 const char* moe_last_error(void);
+
+/* 1 if this library was built with bounds checks (MOE_CHECK_BOUNDS: the file
+ * libmoe_b200_checked.so), else 0.  In that build moe_dispatch and
+ * moe_combine check every expert index and slot they are given against E and
+ * C before they touch a row, skip a choice that is out of range and report
+ * it as MOE_STATUS_BAD_INDEX; the expert-parallel calls always check their
+ * rows (MOE_STATUS_BAD_COUNTS).  A debugging aid for callers that build the
+ * routing arrays themselves: the default build trusts them, as the layer's
+ * own kernels produce them in range. */
+int32_t moe_bounds_checked(void);
 
 /* Limit of every bounded wait inside the library's kernels, in ns, for the
  * launches made after this call by any host thread (process-wide); 0
@@ -195,9 +208,11 @@ int32_t moe_topk_assign(const moe_config* cfg, const float* logits, const int32_
 /* Dispatch (the permutation the Switch router's dispatch tensor encodes,
  * sec. 2.4): xe[e, s, :] = x[t, :] for every kept choice (t, j) with
  * e = expert_idx[t, j], s = slot[t, j].  Rows of xe that no token fills are
- * left untouched.  x [T, d], xe [E, C, d] in cfg->dtype. */
+ * left untouched.  x [T, d], xe [E, C, d] in cfg->dtype.  status: see
+ * moe_bounds_checked (unused by the default build). */
 int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert_idx,
-                     const int32_t* slot, const uint8_t* kept, void* xe, moe_stream_t stream);
+                     const int32_t* slot, const uint8_t* kept, void* xe, int32_t* status,
+                     moe_stream_t stream);
 
 /* Expert FFNs as one grouped computation over the kept rows:
  *   H[e, r, :]  = round(ReLU(xe[e, r, :] . W1[e]^T))   W1 [E, f, d]
@@ -244,7 +259,7 @@ int32_t moe_expert_ffn_ex(const moe_config* cfg, const void* xe, const void* W1,
  * y [T, d] in cfg->dtype. */
 int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert_idx,
                     const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
-                    moe_stream_t stream);
+                    int32_t* status, moe_stream_t stream);
 
 /* The whole layer: router (TOPK) -> gate/top-k or RRE -> slot assignment ->
  * dispatch -> expert FFN -> combine, all on `stream`.  Wr (+ bias) for TOPK,

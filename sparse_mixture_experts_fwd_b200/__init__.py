@@ -16,14 +16,16 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+# MOE_B200_CHECK_BOUNDS=1: load the bounds-checked build (moe_bounds_checked)
+CHECK_BOUNDS = os.environ.get("MOE_B200_CHECK_BOUNDS", "0") == "1"
+LIB_PATH = os.path.join(_PKG, "libmoe_b200_checked.so" if CHECK_BOUNDS else "libmoe_b200.so")
 
 MOE_OK = 0
 ERRORS = {-1: "MOE_ERR_INVALID_ARGUMENT", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_ALIGNMENT",
           -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 ROUTE_TOPK, ROUTE_RRE = 0, 1
-STATUS_TIMEOUT, STATUS_BAD_DOMAIN, STATUS_BAD_COUNTS = 1, 2, 4
+STATUS_TIMEOUT, STATUS_BAD_DOMAIN, STATUS_BAD_COUNTS, STATUS_BAD_INDEX = 1, 2, 4, 8
 FFN_WORKSPACE_ZEROED = 1
 
 # every entry point the header declares, with its ctypes signature
@@ -63,14 +65,15 @@ SIGNATURES = {
     "moe_router": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "moe_topk_assign": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                          _vp], _i32),
-    "moe_dispatch": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "moe_dispatch": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "moe_ffn_workspace_size": ([_PCFG], _sz),
     "moe_expert_ffn": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp], _i32),
     "moe_expert_ffn_ex": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, ctypes.c_uint32, _vp,
                            _vp], _i32),
     "moe_set_wait_limit_ns": ([_u64], None),
     "moe_wait_limit_ns": ([], _u64),
-    "moe_combine": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "moe_combine": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "moe_bounds_checked": ([], _i32),
     "moe_layer_forward": ([_PCFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp],
                           _i32),
     "moe_aux_workspace_size": ([_PCFG], _sz),
@@ -231,12 +234,12 @@ def topk_assign(cfg, logits=None, domain_id=None, out=None, workspace=None, stat
     return o
 
 
-def dispatch(cfg, x, expert_idx, slot, kept, xe=None, stream=None):
+def dispatch(cfg, x, expert_idx, slot, kept, xe=None, status=None, stream=None):
     if xe is None:
         xe = torch.empty(cfg.E, cfg.capacity, cfg.d_model, dtype=x.dtype, device=x.device)
     _check(lib.moe_dispatch(ctypes.byref(cfg), _ptr(x, "x"), _ptr(expert_idx, "expert_idx"),
                             _ptr(slot, "slot"), _ptr(kept, "kept"), _ptr(xe, "xe"),
-                            _stream(stream)), "moe_dispatch")
+                            _ptr(status, "status"), _stream(stream)), "moe_dispatch")
     return xe
 
 
@@ -272,12 +275,12 @@ def expert_ffn(cfg, xe, W1, W2, kept_cnt, H=None, ye=None, workspace=None, statu
     return H, ye
 
 
-def combine(cfg, ye, expert_idx, gate, slot, kept, y=None, stream=None):
+def combine(cfg, ye, expert_idx, gate, slot, kept, y=None, status=None, stream=None):
     if y is None:
         y = torch.empty(cfg.T, cfg.d_model, dtype=ye.dtype, device=ye.device)
     _check(lib.moe_combine(ctypes.byref(cfg), _ptr(ye, "ye"), _ptr(expert_idx, "expert_idx"),
                            _ptr(gate, "gate"), _ptr(slot, "slot"), _ptr(kept, "kept"),
-                           _ptr(y, "y"), _stream(stream)), "moe_combine")
+                           _ptr(y, "y"), _ptr(status, "status"), _stream(stream)), "moe_combine")
     return y
 
 

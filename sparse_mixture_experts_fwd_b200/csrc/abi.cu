@@ -167,6 +167,8 @@ void moe_set_wait_limit_ns(uint64_t ns) {
 
 uint64_t moe_wait_limit_ns(void) { return wait_limit_ns(); }
 
+int32_t moe_bounds_checked(void) { return MOE_CHECK_BOUNDS; }
+
 int32_t moe_capacity(int64_t T, int32_t E, double capacity_factor) {
   if (E < 1 || T < 0 || !(capacity_factor >= 0.0)) return -1;
   const double c = std::floor(static_cast<double>(T) / E * capacity_factor);
@@ -200,6 +202,7 @@ size_t moe_workspace_size(const moe_config* cfg) {
 
 int32_t moe_router(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
                    float* logits, int32_t* status, moe_stream_t stream) {
+  CallRange range_("moe_router");
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   if (cfg->T == 0) return MOE_OK;
@@ -217,6 +220,7 @@ int32_t moe_topk_assign(const moe_config* cfg, const float* logits, const int32_
                         int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
                         int32_t* n_dropped, void* workspace, size_t workspace_bytes,
                         int32_t* status, moe_stream_t stream) {
+  CallRange range_("moe_topk_assign");
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   const bool any_tokens = cfg->T > 0;
@@ -242,7 +246,9 @@ int32_t moe_topk_assign(const moe_config* cfg, const float* logits, const int32_
 }
 
 int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert_idx,
-                     const int32_t* slot, const uint8_t* kept, void* xe, moe_stream_t stream) {
+                     const int32_t* slot, const uint8_t* kept, void* xe, int32_t* status,
+                     moe_stream_t stream) {
+  CallRange range_("moe_dispatch");
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   if (cfg->T == 0 || cfg->capacity == 0) return MOE_OK;
@@ -251,7 +257,8 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert
   MOE_TRY(need_ptr4(slot, "slot"));
   if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
   MOE_TRY(need_ptr(xe, "xe"));
-  return launch_dispatch(*cfg, x, expert_idx, slot, kept, xe, reinterpret_cast<cudaStream_t>(stream));
+  return launch_dispatch(*cfg, x, expert_idx, slot, kept, xe, status,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t moe_ffn_workspace_size(const moe_config* cfg) {
@@ -270,6 +277,7 @@ int32_t moe_expert_ffn_ex(const moe_config* cfg, const void* xe, const void* W1,
                           const int32_t* kept_cnt, void* H, void* ye, void* workspace,
                           size_t workspace_bytes, uint32_t flags, int32_t* status,
                           moe_stream_t stream) {
+  CallRange range_("moe_expert_ffn_ex");
   set_last_error("");
   if (flags & ~static_cast<uint32_t>(MOE_FFN_WORKSPACE_ZEROED))
     return fail(MOE_ERR_INVALID_ARGUMENT, "moe_expert_ffn_ex: unknown flag bits");
@@ -295,7 +303,8 @@ int32_t moe_expert_ffn_ex(const moe_config* cfg, const void* xe, const void* W1,
 
 int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert_idx,
                     const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
-                    moe_stream_t stream) {
+                    int32_t* status, moe_stream_t stream) {
+  CallRange range_("moe_combine");
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   if (cfg->T == 0) return MOE_OK;
@@ -305,7 +314,8 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert
   MOE_TRY(need_ptr4(slot, "slot"));
   if (!kept) return fail(MOE_ERR_INVALID_ARGUMENT, "kept is null");
   MOE_TRY(need_ptr(y, "y"));
-  return launch_combine(*cfg, ye, expert_idx, gate, slot, kept, y, reinterpret_cast<cudaStream_t>(stream));
+  return launch_combine(*cfg, ye, expert_idx, gate, slot, kept, y, status,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t moe_aux_workspace_size(const moe_config* cfg) {
@@ -316,6 +326,7 @@ size_t moe_aux_workspace_size(const moe_config* cfg) {
 int32_t moe_aux_loss(const moe_config* cfg, const float* logits, double alpha, double* out,
                      double* f, double* P, void* workspace, size_t workspace_bytes,
                      moe_stream_t stream) {
+  CallRange range_("moe_aux_loss");
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   if (cfg->mode != MOE_ROUTE_TOPK)
@@ -342,6 +353,7 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
                           const int32_t* domain_id, const void* W1, const void* W2, void* y,
                           void* workspace, size_t workspace_bytes, int32_t* status,
                           void* const* stage_events, moe_stream_t stream) {
+  CallRange range_("moe_layer_forward");
   set_last_error("");
   MOE_TRY(check_cfg(cfg));
   const moe_config& c = *cfg;
@@ -414,7 +426,7 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
   // rows of dropped tokens, so ye is not materialised and no combine runs.
   const bool fused_combine = c.k == 1 && c.dtype == MOE_DTYPE_BF16 && c.T > 0;
   const Top1Out top1{tok_of_row, gate, y};
-  MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, s,
+  MOE_TRY(launch_dispatch(c, x, expert_idx, slot, kept, xe, status, s,
                           dispatch_zeroes ? ffn_sync : nullptr, dispatch_zeroes ? n_sync_words : 0,
                           fused_combine ? y : nullptr));
   MOE_TRY(mark(3));
@@ -423,7 +435,7 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
                           fused_combine ? &top1 : nullptr));
   else MOE_TRY(launch_ffn_f32(c, xe, W1, W2, kept_cnt, H, ye, s));
   MOE_TRY(mark(4));
-  if (!fused_combine) MOE_TRY(launch_combine(c, ye, expert_idx, gate, slot, kept, y, s));
+  if (!fused_combine) MOE_TRY(launch_combine(c, ye, expert_idx, gate, slot, kept, y, status, s));
   return mark(5);
 }
 
@@ -468,6 +480,7 @@ int32_t moe_ep_dispatch(const moe_config* cfg, int32_t rank, int32_t world, cons
                         const int32_t* expert_idx, const int32_t* slot, const uint8_t* kept,
                         const int32_t* cnt_all, void* const* xe_peers, int32_t* local_cnt,
                         int32_t* status, moe_stream_t stream) {
+  CallRange range_("moe_ep_dispatch");
   set_last_error("");
   MOE_TRY(check_ep(cfg, rank, world));
   MOE_TRY(need_ptr4(cnt_all, "cnt_all"));
@@ -491,6 +504,7 @@ int32_t moe_ep_combine(const moe_config* cfg, int32_t rank, int32_t world,
                        const void* const* ye_peers, const int32_t* expert_idx, const float* gate,
                        const int32_t* slot, const uint8_t* kept, const int32_t* cnt_all, void* y,
                        int32_t* status, moe_stream_t stream) {
+  CallRange range_("moe_ep_combine");
   set_last_error("");
   MOE_TRY(check_ep(cfg, rank, world));
   if (cfg->T == 0) return MOE_OK;

@@ -6,11 +6,18 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdint>
 #include <string>
 
 #include "../../include/moe_b200.h"
+
+// 1: dispatch and combine check every expert index and slot they read
+// (the libmoe_b200_checked.so build); 0: they trust them.
+#ifndef MOE_CHECK_BOUNDS
+#define MOE_CHECK_BOUNDS 0
+#endif
 
 namespace moe {
 
@@ -24,6 +31,17 @@ int num_sms();                            // SM count of the current device (cac
 uint64_t wait_limit_ns();                 // limit of every bounded wait, for the next launches
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A named NVTX range around one C-ABI call (host side: from entry to return,
+// i.e. validation and enqueueing), so a profiler's timeline shows which call
+// launched which kernels and `ncu --nvtx --nvtx-include` can select them.
+// Without an attached tool it costs one branch.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // Launch `kern` with programmatic stream serialisation (see pdl_wait).
 template <typename... KArgs, typename... Args>
@@ -96,7 +114,8 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
 // zero_words (nullable): n_zero words the dispatch kernel clears for the next kernel;
 // y_zero (nullable): y [T, d], whose rows of tokens with no kept choice it zeroes
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
-                        const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
+                        const int32_t* slot, const uint8_t* kept, void* xe, int32_t* status,
+                        cudaStream_t s,
                         unsigned int* zero_words = nullptr, int n_zero = 0,
                         void* y_zero = nullptr);
 // Switch load-balancing loss (eqs. 4-6) and routing entropy from logits [T, E]
@@ -105,7 +124,7 @@ int32_t launch_aux_loss(const moe_config& c, const float* logits, double alpha, 
                         double* f, double* P, void* workspace, cudaStream_t s);
 int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* expert_idx,
                        const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
-                       cudaStream_t s);
+                       int32_t* status, cudaStream_t s);
 // expert parallelism over the ranks of one node: the receive buffers of all
 // ranks as mapped into this process, rank order
 constexpr int kMaxEpRanks = 8;

@@ -31,15 +31,27 @@
 namespace moe {
 namespace {
 
+// A kept choice's expert and slot inside [0, E) x [0, C).  The bounds-checked
+// build tests them before a row is touched; the default build trusts them.
+__device__ __forceinline__ bool choice_in_range(int e, int s, int E, int C) {
+#if MOE_CHECK_BOUNDS
+  return e >= 0 && e < E && s >= 0 && s < C;
+#else
+  (void)e; (void)s; (void)E; (void)C;
+  return true;
+#endif
+}
+
 template <int K>
-__global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, int C,
+__global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, int E, int C,
                                                        const uint4* __restrict__ x,
                                                        const int32_t* __restrict__ expert_idx,
                                                        const int32_t* __restrict__ slot,
                                                        const uint8_t* __restrict__ kept,
                                                        uint4* __restrict__ xe,
                                                        unsigned int* __restrict__ zero_words,
-                                                       int n_zero, uint4* __restrict__ y_zero) {
+                                                       int n_zero, uint4* __restrict__ y_zero,
+                                                       int32_t* __restrict__ status) {
   dev::pdl_trigger();
   dev::pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -47,6 +59,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
   // counters the next kernel on this stream expects at zero (the fused expert FFN)
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0u;
+  bool bad = false;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
        t += nwarps) {
     int64_t dst0 = 0, dst1 = 0;  // the kept choices' xe rows, in choice order
@@ -54,8 +67,12 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
 #pragma unroll
     for (int j = 0; j < K; ++j) {
       if (__ldg(kept + t * K + j)) {
-        const int64_t d = (static_cast<int64_t>(__ldg(expert_idx + t * K + j)) * C +
-                           __ldg(slot + t * K + j)) * row_vec;
+        const int e = __ldg(expert_idx + t * K + j), sl = __ldg(slot + t * K + j);
+        if (!choice_in_range(e, sl, E, C)) {
+          bad = true;
+          continue;
+        }
+        const int64_t d = (static_cast<int64_t>(e) * C + sl) * row_vec;
         if (nd == 0) dst0 = d;
         else dst1 = d;
         ++nd;
@@ -76,6 +93,7 @@ __global__ void __launch_bounds__(256) dispatch_kernel(int64_t T, int row_vec, i
       if (K == 2 && nd == 2) xe[dst1 + v] = val;
     }
   }
+  if (MOE_CHECK_BOUNDS && bad && lane == 0 && status) atomicOr(status, MOE_STATUS_BAD_INDEX);
 }
 
 struct Bf16x8 {
@@ -113,18 +131,20 @@ struct F32x4 {
 };
 
 template <int K, class V>
-__global__ void __launch_bounds__(256) combine_kernel(int64_t T, int row_vec, int C,
+__global__ void __launch_bounds__(256) combine_kernel(int64_t T, int row_vec, int E, int C,
                                                       const uint4* __restrict__ ye,
                                                       const int32_t* __restrict__ expert_idx,
                                                       const float* __restrict__ gate,
                                                       const int32_t* __restrict__ slot,
                                                       const uint8_t* __restrict__ kept,
-                                                      uint4* __restrict__ y) {
+                                                      uint4* __restrict__ y,
+                                                      int32_t* __restrict__ status) {
   dev::pdl_trigger();
   dev::pdl_wait();
   constexpr int N = V::kN;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  bool bad = false;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
        t += nwarps) {
     int64_t src[K];
@@ -133,8 +153,12 @@ __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int row_vec, in
 #pragma unroll
     for (int j = 0; j < K; ++j) {
       if (__ldg(kept + t * K + j)) {
-        src[ns] = (static_cast<int64_t>(__ldg(expert_idx + t * K + j)) * C +
-                   __ldg(slot + t * K + j)) * row_vec;
+        const int e = __ldg(expert_idx + t * K + j), sl = __ldg(slot + t * K + j);
+        if (!choice_in_range(e, sl, E, C)) {
+          bad = true;
+          continue;
+        }
+        src[ns] = (static_cast<int64_t>(e) * C + sl) * row_vec;
         g[ns] = __ldg(gate + t * K + j);
         ++ns;
       }
@@ -162,6 +186,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int64_t T, int row_vec, in
       dst[v] = V::pack(acc);
     }
   }
+  if (MOE_CHECK_BOUNDS && bad && lane == 0 && status) atomicOr(status, MOE_STATUS_BAD_INDEX);
 }
 
 unsigned grid_for_tokens(int64_t T) {
@@ -336,26 +361,26 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(
 }  // namespace
 
 int32_t launch_dispatch(const moe_config& c, const void* x, const int32_t* expert_idx,
-                        const int32_t* slot, const uint8_t* kept, void* xe, cudaStream_t s,
-                        unsigned int* zero_words, int n_zero, void* y_zero) {
+                        const int32_t* slot, const uint8_t* kept, void* xe, int32_t* status,
+                        cudaStream_t s, unsigned int* zero_words, int n_zero, void* y_zero) {
   if (c.T == 0 || (c.capacity == 0 && !y_zero)) return MOE_OK;
   const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
   const unsigned grid = grid_for_tokens(c.T);
   uint4* yz = static_cast<uint4*>(y_zero);
   if (c.k == 1)
-    launch_pdl(dispatch_kernel<1>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity,
+    launch_pdl(dispatch_kernel<1>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, c.capacity,
                static_cast<const uint4*>(x), expert_idx, slot, kept, static_cast<uint4*>(xe),
-               zero_words, n_zero, yz);
+               zero_words, n_zero, yz, status);
   else
-    launch_pdl(dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity,
+    launch_pdl(dispatch_kernel<2>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, c.capacity,
                static_cast<const uint4*>(x), expert_idx, slot, kept, static_cast<uint4*>(xe),
-               zero_words, n_zero, yz);
+               zero_words, n_zero, yz, status);
   return check_launch("dispatch_kernel");
 }
 
 int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* expert_idx,
                        const float* gate, const int32_t* slot, const uint8_t* kept, void* y,
-                       cudaStream_t s) {
+                       int32_t* status, cudaStream_t s) {
   if (c.T == 0) return MOE_OK;
   const int row_vec = static_cast<int>(c.d_model * elem_size(c.dtype) / 16);
   const unsigned grid = grid_for_tokens(c.T);
@@ -363,18 +388,18 @@ int32_t launch_combine(const moe_config& c, const void* ye, const int32_t* exper
   uint4* yv = static_cast<uint4*>(y);
   if (c.dtype == MOE_DTYPE_BF16) {
     if (c.k == 1)
-      launch_pdl(combine_kernel<1, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
-                                                     gate, slot, kept, yv);
+      launch_pdl(combine_kernel<1, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, c.capacity, yev, expert_idx,
+                                                     gate, slot, kept, yv, status);
     else
-      launch_pdl(combine_kernel<2, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
-                                                     gate, slot, kept, yv);
+      launch_pdl(combine_kernel<2, Bf16x8>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, c.capacity, yev, expert_idx,
+                                                     gate, slot, kept, yv, status);
   } else {
     if (c.k == 1)
-      launch_pdl(combine_kernel<1, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
-                                                    gate, slot, kept, yv);
+      launch_pdl(combine_kernel<1, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, c.capacity, yev, expert_idx,
+                                                    gate, slot, kept, yv, status);
     else
-      launch_pdl(combine_kernel<2, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.capacity, yev, expert_idx,
-                                                    gate, slot, kept, yv);
+      launch_pdl(combine_kernel<2, F32x4>, dim3(grid), dim3(256), 0, s, c.T, row_vec, c.E, c.capacity, yev, expert_idx,
+                                                    gate, slot, kept, yv, status);
   }
   return check_launch("combine_kernel");
 }

@@ -174,6 +174,7 @@ extern "C" int32_t sparseclip_norm(const float* const* dense, const int64_t* den
                                    const int64_t* sparse_len, int32_t n_sparse,
                                    int32_t num_experts, double* out, void* workspace,
                                    size_t workspace_bytes, moe_stream_t stream) {
+  CallRange range_("sparseclip_norm");
   set_last_error("");
   if (n_dense < 0 || n_sparse < 0 || static_cast<int64_t>(n_dense) + n_sparse > kMaxSegs)
     return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_norm: segment counts out of range");
@@ -220,6 +221,7 @@ extern "C" int32_t sparseclip_clip(float* const* dense, const int64_t* dense_len
                                    int32_t n_sparse, int32_t num_experts, double max_norm,
                                    double* out, void* workspace, size_t workspace_bytes,
                                    moe_stream_t stream) {
+  CallRange range_("sparseclip_clip");
   set_last_error("");
   if (!(max_norm > 0.0) || !std::isfinite(max_norm))
     return fail(MOE_ERR_INVALID_ARGUMENT, "sparseclip_clip: max_norm must be positive and finite");

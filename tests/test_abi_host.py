@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(moe):
 
 
 def test_struct_layout(moe):
-    assert moe.lib.moe_abi_version() == 2
+    assert moe.lib.moe_abi_version() == 3
     assert moe.lib.moe_config_size() == 56 == ctypes.sizeof(moe.MoEConfig)
     assert moe.lib.moe_workspace_map_size() == ctypes.sizeof(moe.WorkspaceMap)
 
@@ -110,7 +110,7 @@ def test_calls_rejected_on_host(moe):
     # bf16 expert FFN without its tile-counter workspace
     assert moe.lib.moe_expert_ffn(ctypes.byref(c), p, p, p, p, p, p, None, 0, None, None) == -4
     assert moe.lib.moe_ffn_workspace_size(ctypes.byref(c)) == 768  # 4 * (1 + 128) -> 256-aligned
-    assert moe.lib.moe_dispatch(None, p, p, p, p, p, None) == -1
+    assert moe.lib.moe_dispatch(None, p, p, p, p, p, None, None) == -1
     # sparseclip
     assert moe.lib.sparseclip_norm(None, None, 0, None, None, 0, 0, p, p, 1 << 20, None) == -1
     assert moe.lib.sparseclip_workspace_size(1, 64) == 1024 * 2 * 8
