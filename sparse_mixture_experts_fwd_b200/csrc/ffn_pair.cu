@@ -413,16 +413,20 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
+      // CTA 0 takes each tile one tile ahead: the counter's atomic round trip
+      // then runs under the current tile's loads instead of between tiles
+      unsigned int taken = rank == 0 ? atomicAdd(p.tile_ctr, 1u) : 0u;
       while (!ab.raised()) {
         int t;
         if (rank == 0) {
-          t = static_cast<int>(atomicAdd(p.tile_ctr, 1u));
+          t = static_cast<int>(taken);
           if (t < 0 || t >= total) t = -1;  // (negative only from a counter not zeroed)
           if (!mbar_wait_cluster(&ring_empty[slot], rphase ^ 1u, ab)) break;
           s_ring[slot] = t;
           st_cluster_u32(mapa(&s_ring[slot], 1), t);
           dev::mbar_arrive(&ring_full[slot]);
           mbar_arrive_cluster(mapa(&ring_full[slot], 1));
+          if (t >= 0) taken = atomicAdd(p.tile_ctr, 1u);  // used at the next iteration
         } else {
           if (!mbar_wait_cluster(&ring_full[slot], rphase, ab)) break;
           t = s_ring[slot];
@@ -447,23 +451,19 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
           if (!wait_count(p.chunk_ctr + x.e * p.maxc + x.c, need, ab)) break;
           fence_proxy_async_global();  // generic-proxy H stores -> async-proxy (TMA) reads
         }
-        const uint32_t tx = static_cast<uint32_t>(2 * (kABytes + half * kBK * 2));
+        // the token half is one box of the smallest of 128/64/32/16/8 rows that
+        // holds it: one TMA per operand and stage (rows past the chunk load
+        // but no MMA reads them)
+        int box = 0;
+        while (box + 1 < kBoxes && (kHalf >> (box + 1)) >= half) ++box;
+        const uint32_t tx = static_cast<uint32_t>(2 * (kABytes + (kHalf >> box) * kBK * 2));
         bool ok = true;
         for (int kb = 0; kb < K / kBK; ++kb) {
           if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, ab)) { ok = false; break; }
           if (rank == 0) dev::mbar_arrive_expect_tx(&full_bar[stage], tx);
           const uint32_t full0 = mapa(&full_bar[stage], 0);
           tma_load_2d_pair(smA + stage * kABytes, ta, full0, kb * kBK, a_row);
-          uint8_t* dstB = smB + stage * kBBytesMax;
-          int done = 0;
-#pragma unroll
-          for (int i = 0; i < kBoxes; ++i) {
-            const int rows = kHalf >> i;
-            if (half - done >= rows) {
-              tma_load_2d_pair(dstB + done * (kBK * 2), tb + i, full0, kb * kBK, b_row + done);
-              done += rows;
-            }
-          }
+          tma_load_2d_pair(smB + stage * kBBytesMax, tb + box, full0, kb * kBK, b_row);
           ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -773,10 +773,13 @@ int32_t launch_ffn_pair_fused(const moe_config& c, const void* xe, const void* W
   if (cudaOccupancyMaxActiveClusters(&resident, ffn_pair_kernel, &cfg) != cudaSuccess ||
       resident < 1)
     return check_launch("cudaOccupancyMaxActiveClusters(ffn_pair_kernel)");
-  // lag: GEMM-2 tiles of expert e follow about two waves of GEMM-1 tiles of later experts
-  const int64_t g1_per_expert = static_cast<int64_t>(p.nm1) * maxc;
+  // lag: the GEMM-2 tiles of expert e come after the GEMM-1 tiles of the next
+  // L experts, about three tiles per pair (each pair holds up to three tiles
+  // between taking one and finishing its epilogue), so their wait for H is
+  // normally over when they are taken; chunks per expert estimated as C / 256
+  const int64_t g1_per_expert = std::max<int64_t>(1, static_cast<int64_t>(p.nm1) * C / kMaxN);
   p.lag = static_cast<int>(std::min<int64_t>(
-      E, std::max<int64_t>(1, (2 * static_cast<int64_t>(resident) + g1_per_expert - 1) /
+      E, std::max<int64_t>(1, (3 * static_cast<int64_t>(resident) + g1_per_expert - 1) /
                                   g1_per_expert)));
   const int64_t max_tiles = E * static_cast<int64_t>(maxc) * (p.nm1 + p.nm2);
   if (max_tiles > 2147483647) return fail(MOE_ERR_UNSUPPORTED, "ffn_pair_kernel: too many tiles");
