@@ -250,7 +250,7 @@ def kernel_launches(w, C):
         route = 3                       # fp32 router, gate/top-k, slot assignment
     # bf16: one persistent kernel for both GEMMs when C <= 128 (single CTAs) or
     # C >= 512 (SM pairs); two grouped launches in between; fp32: two FMA GEMMs
-    ffn = 1 if (bf16 and (C <= 128 or C >= 512)) else 2
+    ffn = 1 if (bf16 and (C <= 128 or (C >= 512 and w.d_model >= 2048))) else 2
     combine = 0 if (bf16 and w.k == 1) else 1   # top-1 bf16: inside the FFN's GEMM 2
     return route + 1 + ffn + combine
 
@@ -429,7 +429,9 @@ def run_b200(args, w, world, rank, local):
         "grouped_gemm_f32_kernel x2" if w.dtype == "f32" else
         "ffn_tc_kernel x1 (both GEMMs fused)" if C <= 128 else
         "gemm_tc_kernel x2 (H = ReLU(xe W1^T), ye = H W2^T)" if C < 512 else
-        "ffn_pair_kernel x1 on SM pairs (both GEMMs fused, tokens on the MMA's N side)"))
+        "ffn_pair_kernel x1 on SM pairs (both GEMMs fused, tokens on the MMA's N side)"
+        if w.d_model >= 2048 else
+        "gemm_pair_kernel x2 on SM pairs (H = ReLU(xe W1^T), ye = H W2^T)"))
     roof["peak_source"] = peaks["source"]
     roof["algorithmic_per_launch"] = (f"{ffn_bytes / 1e9:.4f} GB" if roof["bound"] == "hbm"
                                       else f"{ffn_flops / 1e12:.4f} TFLOP")

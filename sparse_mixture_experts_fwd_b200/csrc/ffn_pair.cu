@@ -6,36 +6,42 @@
 //
 // Orientation: the weights are the MMA's M side and the tokens its N side.
 // A tile is 256 output features (W1 or W2 rows) x N tokens of one expert,
-// N <= 256 in steps of 16: an expert's r kept rows are cut into
-// ceil(r / 256) chunks of equal size rounded up to 16, so an expert with 530
-// rows computes 544 token columns instead of three 256-row blocks (768).
-// CTA r of the pair holds features [128r, 128r + 128) of the tile (its half
-// of the A operand) and tokens [rN/2, rN/2 + N/2) of the chunk (its half of
-// B); its TMEM lanes are its 128 features and the columns the N tokens.  The
-// token half is fetched as up to four TMA boxes of 128/64/32/16/8 rows, so no
-// byte past the chunk is loaded.
-//
+// N <= 256 in steps of 16: an expert's r kept rows are cut into chunks of 256
+// rows and one of the rest, rounded up to 16, so an expert with 530 rows
+// computes 544 token columns instead of three 256-row blocks (768).  CTA r
+// of the pair holds features [128r, 128r + 128) of the tile (its half of the
+// A operand) and tokens [rN/2, rN/2 + N/2) of the chunk (its half of B); its
+// TMEM lanes are its 128 features and the columns the N tokens.  The token
+// half is fetched as one TMA box of 128, 64, 32, 16 or 8 rows, the smallest
+// that holds it (one load per operand and stage: more, smaller boxes per
+// stage left the MMAs waiting on the TMA unit).
+
 // Both GEMMs run in one tile sequence of "units" (unit u: the GEMM-1 tiles
 // of expert u, then the GEMM-2 tiles of expert u - L), tiles of one expert
 // ordered (feature block, chunk) so the chunks sharing a weight tile run side
-// by side and read it from L2.  CTA 0 of each pair takes the next tile from a
-// global counter and hands it to CTA 1 through a shared-memory ring in the
-// cluster, so the load balances to within one tile, there is no tail between
-// the GEMMs and a pair that is not yet running holds no tile.  A GEMM-2 tile
-// of (expert, chunk) needs every GEMM-1 tile of that chunk: each epilogue warp
-// that stored its 32 features of a GEMM-1 tile adds one (release) to the
-// chunk's counter, and the producers of a GEMM-2 tile wait (acquire, bounded)
-// for 8 per GEMM-1 feature block.  H of the experts in flight stays in L2.
+// by side and read it from L2.  CTA 0 of each pair takes tiles from a global
+// counter one tile ahead and publishes each to both CTAs through a
+// shared-memory ring in the cluster one tile before its loads begin, so the
+// load balances to within one tile, there is no tail between the GEMMs and a
+// pair that is not yet running holds no tile.  A GEMM-2 tile of (expert,
+// chunk) needs every GEMM-1 tile of that chunk: each epilogue warp that
+// stored its part of a GEMM-1 tile adds one (release) to the chunk's counter,
+// and the producers of a GEMM-2 tile wait (acquire, bounded) for 16 per
+// GEMM-1 feature block.  H of the experts in flight stays in L2.
 //
 // Epilogue: an accumulator column is one token, a lane one feature, so each
-// warp pairs neighbouring features with one shuffle and stores 4 bytes per
-// lane: every store instruction writes two 64-byte runs of two token rows.
-// GEGLU: lanes 2i, 2i + 1 hold hidden unit i's gate and linear parts.
-// Top-1 layers: GEMM 2 writes gate * row straight to y in token order.
-//
-// Roles per CTA (192 threads): warp 0 lane 0 loads this CTA's halves (CTA 0's
+// warp packs a lane's two tokens into a bf16x2 word, swaps it with the
+// neighbour lane and stores 4 bytes per lane: every store instruction writes
+// two 64-byte runs of two token rows.  GEGLU: lanes 2i, 2i + 1 hold hidden
+// unit i's gate and linear parts.  Top-1 layers: GEMM 2 writes gate * row
+// straight to y in token order.  Two accumulators in tensor memory let a
+// tile's epilogue run under the next tile's MMAs; eight warps (two per lane
+// quarter, alternate 32-column blocks) keep it shorter than a short-K tile's
+// main loop.
+
+// Roles per CTA (320 threads): warp 0 lane 0 loads this CTA's halves (CTA 0's
 // also takes tiles); warp 1 lane 0 of CTA 0 issues the MMAs (M = 256) and
-// commits them to both CTAs; warps 2-5 drain their CTA's TMEM.  Every wait is
+// commits them to both CTAs; warps 2-9 drain their CTA's TMEM.  Every wait is
 // bounded and shares the call's give-up signal; TMA loads fill only the
 // issuing CTA's shared memory (no multicast).
 #include <cuda.h>
@@ -48,24 +54,25 @@
 namespace moe {
 namespace {
 
-constexpr int kHalf = 128;                // A rows (features) per CTA
-constexpr int kBM = 256;                  // features per tile
-constexpr int kMaxN = 256;                // tokens per tile
-constexpr int kNStep = 16;                // token granularity of a tile
+constexpr int kHalf = 128;                 // A rows (features) per CTA
+constexpr int kBM = 256;                   // features per tile
+constexpr int kMaxN = 256;                 // tokens per tile (one accumulator)
+constexpr int kChunk = kMaxN;              // rows per chunk of an expert
 constexpr int kBK = 64, kUmmaK = 16;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;               // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kStages = 6;
 constexpr int kRing = 8;
-constexpr int kABytes = kHalf * kBK * 2;         // 16 KB
-constexpr int kBBytesMax = (kMaxN / 2) * kBK * 2;  // 16 KB
+constexpr int kABytes = kHalf * kBK * 2;          // 16 KB
+constexpr int kBRowsMax = kMaxN / 2;              // token rows per CTA
+constexpr int kBBytesMax = kBRowsMax * kBK * 2;   // 16 KB
 constexpr int kStageBytes = kABytes + kBBytesMax;
 constexpr int kTmemCols = 512;
-constexpr int kAccStride = 256;
 constexpr int kMaxE = 256;
 constexpr int kMaxUnits = 2 * kMaxE;
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
 constexpr int kBoxes = 5;                 // token-row boxes of 128, 64, 32, 16, 8 rows
-constexpr int kCtrPerTile = 8;            // counter arrivals per GEMM-1 tile: 4 warps x 2 CTAs
+constexpr int kCtrPerTile = 2 * kEpiWarps;  // counter arrivals per GEMM-1 tile: both CTAs' warps
 
 struct Maps {
   CUtensorMap w1;           // W1 [E * n1, d], box 128 x 64
@@ -89,6 +96,23 @@ struct PairParams {
   const float* gate;
   __nv_bfloat16* y;
 };
+
+// Shape of the tile of chunk c of an expert with r kept rows: N columns, the
+// first N / 2 rows in CTA 0's half of B, the rest in CTA 1's.
+struct Geo {
+  int row0;   // first row of the chunk within the expert
+  int rows;   // rows (tokens) of the chunk
+  int N;      // MMA N
+  int half;   // token rows per CTA (B operand)
+};
+MOE_DEV Geo chunk_geo(int r, int c) {
+  Geo g;
+  g.row0 = c * kChunk;
+  g.rows = min(kChunk, r - g.row0);
+  g.N = (g.rows + 15) / 16 * 16;
+  g.half = g.N / 2;
+  return g;
+}
 
 struct Tile {
   int kind;  // 1: GEMM 1, 2: GEMM 2
@@ -249,75 +273,80 @@ MOE_DEV bool wait_count(const unsigned int* p, unsigned int need, const dev::Abo
   }
 }
 
-MOE_DEV uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
+
+// bf16x2 of (lo, hi) rounded to nearest even, lo in the low half; RELU also
+// clamps each to >= 0 (cvt's .relu: the rounding keeps the sign, so it is the
+// same as clamping first)
+template <bool RELU>
+MOE_DEV uint32_t cvt_pair(float lo, float hi) {
+  uint32_t d;
+  if (RELU)
+    asm("cvt.rn.relu.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  else
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
 }
 
 // Stores one 32-lane x NC-column accumulator block of a ReLU / plain tile:
-// lane = feature fe0 + lane, column j = token n0 + j.  Lanes 2i and 2i + 1
-// swap one value per token pair, so lane 2i stores features (2i, 2i + 1) of
-// token 2j and lane 2i + 1 those of token 2j + 1, 4 bytes each.
+// lane = feature fe0 + lane, column n0 + j = chunk row n0 + j.  Each lane
+// packs its feature at rows (2j, 2j + 1) into one bf16x2 word and trades it
+// with its neighbour lane, so lane 2i stores features (2i, 2i + 1) of row 2j
+// and lane 2i + 1 those of row 2j + 1, 4 bytes each.
 template <int NC, bool RELU, bool SCATTER>
-MOE_DEV void store_pairs(const uint32_t (&r)[32], int lane, int n0, int rows_valid,
+MOE_DEV void store_pairs(const uint32_t (&r)[32], int lane, const Geo& g, int n0,
                          __nv_bfloat16* out, int64_t row_base, int64_t ld, int fe, bool fe_ok,
                          int tok_lane, float g_lane) {
   const int p = lane & 1;
 #pragma unroll
   for (int j = 0; j < NC / 2; ++j) {
-    const float mine0 = __uint_as_float(r[2 * j]), mine1 = __uint_as_float(r[2 * j + 1]);
-    const float other = __shfl_xor_sync(0xffffffffu, p ? mine0 : mine1, 1);
-    float lo = p ? other : mine0;
-    float hi = p ? mine1 : other;
-    const int n = n0 + 2 * j + p;
+    float v0 = __uint_as_float(r[2 * j]), v1 = __uint_as_float(r[2 * j + 1]);
     int tok = 0;
-    float g = 1.f;
     if (SCATTER) {
+      v0 *= __shfl_sync(0xffffffffu, g_lane, 2 * j);
+      v1 *= __shfl_sync(0xffffffffu, g_lane, 2 * j + 1);
       tok = __shfl_sync(0xffffffffu, tok_lane, 2 * j + p);
-      g = __shfl_sync(0xffffffffu, g_lane, 2 * j + p);
-      lo *= g;
-      hi *= g;
     }
-    if (RELU) {
-      lo = fmaxf(lo, 0.f);
-      hi = fmaxf(hi, 0.f);
-    }
-    if (fe_ok && n < rows_valid) {
-      const int64_t row = SCATTER ? static_cast<int64_t>(tok) : row_base + n;
-      *reinterpret_cast<uint32_t*>(out + row * ld + fe) = pack_bf16(lo, hi);
+    const uint32_t mine = cvt_pair<RELU>(v0, v1);          // my feature, columns 2j | 2j+1
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+    // even lane: (mine.lo, other.lo) = column 2j; odd lane: (other.hi, mine.hi) = column 2j+1
+    const uint32_t w = p ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
+    const int row = n0 + 2 * j + p;
+    if (fe_ok && row < g.rows) {
+      const int64_t orow = SCATTER ? static_cast<int64_t>(tok) : row_base + row;
+      *reinterpret_cast<uint32_t*>(out + orow * ld + fe) = w;
     }
   }
 }
 
 // GEGLU GEMM-1 block: lanes 4k, 4k + 1 hold hidden unit 2k's gate and linear
 // rows, lanes 4k + 2, 4k + 3 unit 2k + 1's.  Even lanes form GELU(g) * l of
-// the even tokens, odd lanes of the odd tokens; then lanes L and L ^ 2 trade
-// values so that each stores units (2k, 2k + 1) of one token in 4 bytes.
+// the even columns, odd lanes of the odd ones; then lanes L and L ^ 2 trade
+// values so that each stores units (2k, 2k + 1) of one row in 4 bytes.
 template <int NC>
-MOE_DEV void store_geglu(const uint32_t (&r)[32], int lane, int n0, int rows_valid,
+MOE_DEV void store_geglu(const uint32_t (&r)[32], int lane, const Geo& g, int n0,
                          __nv_bfloat16* out, int64_t row_base, int64_t ld, int unit_even,
                          bool unit_ok) {
-  const int p = lane & 1;        // token parity this lane finishes
+  const int p = lane & 1;        // column parity this lane finishes
   const int s = (lane >> 1) & 1; // 0: unit 2k, 1: unit 2k + 1
   float h[NC / 2];
 #pragma unroll
   for (int j = 0; j < NC / 2; ++j) {
-    // lane 2i (gate) needs the linear part of token 2j, lane 2i + 1 the gate of token 2j + 1
+    // lane 2i (gate) needs the linear part of column 2j, lane 2i + 1 the gate of column 2j + 1
     const float mine0 = __uint_as_float(r[2 * j]), mine1 = __uint_as_float(r[2 * j + 1]);
     const float other = __shfl_xor_sync(0xffffffffu, p ? mine0 : mine1, 1);
-    const float g = p ? other : mine0;
+    const float gt = p ? other : mine0;
     const float l = p ? mine1 : other;
-    h[j] = dev::geglu(g, l);  // unit u(lane) at token 2j + p
+    h[j] = dev::geglu(gt, l);  // unit u(lane) at column 2j + p
   }
 #pragma unroll
   for (int i = 0; i < NC / 4; ++i) {
     const float send = s ? h[2 * i] : h[2 * i + 1];
     const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-    const float u0 = s ? recv : h[2 * i];          // unit 2k at the stored token
-    const float u1 = s ? h[2 * i + 1] : recv;      // unit 2k + 1
-    const int n = n0 + 4 * i + 2 * s + p;
-    if (unit_ok && n < rows_valid)
-      *reinterpret_cast<uint32_t*>(out + (row_base + n) * ld + unit_even) = pack_bf16(u0, u1);
+    const uint32_t w = cvt_pair<false>(s ? recv : h[2 * i],       // unit 2k
+                                       s ? h[2 * i + 1] : recv);  // unit 2k + 1
+    const int row = n0 + 4 * i + 2 * s + p;
+    if (unit_ok && row < g.rows)
+      *reinterpret_cast<uint32_t*>(out + (row_base + row) * ld + unit_even) = w;
   }
 }
 
@@ -328,7 +357,7 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
   __shared__ uint64_t ring_full[kRing], ring_empty[kRing];
   __shared__ int s_ring[kRing];
   __shared__ uint32_t s_tmem_base;
-  __shared__ int s_rows[kMaxE], s_nc[kMaxE], s_base[kMaxE], s_prefix[kMaxUnits + 1];
+  __shared__ int s_rows[kMaxE], s_nc[kMaxE], s_prefix[kMaxUnits + 1];
   __shared__ volatile int s_abort;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -356,12 +385,12 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
     }
     for (int a = 0; a < 2; ++a) {
       dev::mbar_init(&tfull_bar[a], 1);
-      dev::mbar_init(&tempty_bar[a], 2 * 128);  // epilogue threads of both CTAs (CTA 0's used)
+      dev::mbar_init(&tempty_bar[a], 2 * 32 * kEpiWarps);  // epilogue threads of both CTAs (CTA 0's used)
     }
     for (int r = 0; r < kRing; ++r) {
       dev::mbar_init(&ring_full[r], 1);
-      // CTA 0's: its MMA lane and 4 epilogue warps, CTA 1's producer and 4 epilogue warps
-      dev::mbar_init(&ring_empty[r], 10);
+      // CTA 0's: its MMA lane and epilogue warps, CTA 1's producer and epilogue warps
+      dev::mbar_init(&ring_empty[r], 2 + 2 * kEpiWarps);
     }
     dev::mbar_init(&done_bar, 1);
     dev::fence_mbar_init();
@@ -378,13 +407,8 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
   for (int e = tid; e < E; e += kThreads) {
     int r = p.kept_cnt[e];
     r = r < 0 ? 0 : (r > p.C ? p.C : r);
-    // chunks of at most 256 rows, equal sizes rounded up to 16
-    const int nc0 = (r + kMaxN - 1) / kMaxN;
-    int base = nc0 ? (r + nc0 - 1) / nc0 : 0;
-    base = (base + kNStep - 1) / kNStep * kNStep;
     s_rows[e] = r;
-    s_base[e] = base;
-    s_nc[e] = base ? (r + base - 1) / base : 0;
+    s_nc[e] = (r + kChunk - 1) / kChunk;  // chunks of 256 rows, the last one the rest
   }
   __syncthreads();
   if (tid == 0) {
@@ -408,55 +432,72 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
   if (warp == 0) {
     // ---------------- tile taker (CTA 0) + TMA producer (both CTAs) ----------------
     if (lane == 0) {
-      int slot = 0;
+      int slot = 0;            // CTA 1: next ring slot to read
       uint32_t rphase = 0;
+      int pslot = 0;           // CTA 0: next ring slot to write
+      uint32_t pphase = 0;
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      // CTA 0 takes each tile one tile ahead: the counter's atomic round trip
-      // then runs under the current tile's loads instead of between tiles
-      unsigned int taken = rank == 0 ? atomicAdd(p.tile_ctr, 1u) : 0u;
-      while (!ab.raised()) {
+      // CTA 0 publishes each tile one tile before it loads it, and takes it
+      // from the counter one tile before that: CTA 1 starts its loads of a
+      // tile as early as CTA 0, and no atomic round trip sits between tiles
+      auto clamp_tile = [&](unsigned int v) {
+        const int t = static_cast<int>(v);
+        return (t < 0 || t >= total) ? -1 : t;  // (negative only from a counter not zeroed)
+      };
+      auto publish = [&](int t) -> bool {
+        if (!mbar_wait_cluster(&ring_empty[pslot], pphase ^ 1u, ab)) return false;
+        s_ring[pslot] = t;
+        st_cluster_u32(mapa(&s_ring[pslot], 1), t);
+        dev::mbar_arrive(&ring_full[pslot]);
+        mbar_arrive_cluster(mapa(&ring_full[pslot], 1));
+        if (++pslot == kRing) { pslot = 0; pphase ^= 1u; }
+        return true;
+      };
+      int cur = -1;
+      unsigned int pending = 0u;
+      bool run = true;
+      if (rank == 0) {
+        cur = clamp_tile(atomicAdd(p.tile_ctr, 1u));
+        run = publish(cur);
+        if (cur >= 0) pending = atomicAdd(p.tile_ctr, 1u);
+      }
+      while (run && !ab.raised()) {
         int t;
         if (rank == 0) {
-          t = static_cast<int>(taken);
-          if (t < 0 || t >= total) t = -1;  // (negative only from a counter not zeroed)
-          if (!mbar_wait_cluster(&ring_empty[slot], rphase ^ 1u, ab)) break;
-          s_ring[slot] = t;
-          st_cluster_u32(mapa(&s_ring[slot], 1), t);
-          dev::mbar_arrive(&ring_full[slot]);
-          mbar_arrive_cluster(mapa(&ring_full[slot], 1));
-          if (t >= 0) taken = atomicAdd(p.tile_ctr, 1u);  // used at the next iteration
+          t = cur;
+          if (t < 0) break;
+          const int nxt = clamp_tile(pending);  // taken one tile ago
+          if (!publish(nxt)) break;
+          if (nxt >= 0) pending = atomicAdd(p.tile_ctr, 1u);
+          cur = nxt;
         } else {
           if (!mbar_wait_cluster(&ring_full[slot], rphase, ab)) break;
           t = s_ring[slot];
           mbar_arrive_cluster(ring_empty0 + static_cast<uint32_t>(slot) * ring_stride);
+          if (++slot == kRing) { slot = 0; rphase ^= 1u; }
         }
-        if (++slot == kRing) { slot = 0; rphase ^= 1u; }
         if (t < 0) break;
         const Tile x = sc.decode(t);
-        const int base = s_base[x.e];
-        const int row0 = x.c * base;
-        const int rows_c = min(base, s_rows[x.e] - row0);
-        const int N = (rows_c + kNStep - 1) / kNStep * kNStep;
-        const int half = N / 2;  // token rows of this CTA (multiple of 8)
+        const Geo g = chunk_geo(s_rows[x.e], x.c);
         const CUtensorMap* ta = x.kind == 1 ? &maps.w1 : &maps.w2;
         const CUtensorMap* tb = x.kind == 1 ? maps.x : maps.h;
         const int K = x.kind == 1 ? p.d : p.f;
         const int a_row = x.e * (x.kind == 1 ? p.n1 : p.d) + x.m * kBM + static_cast<int>(rank) * kHalf;
-        const int b_row = x.e * p.C + row0 + static_cast<int>(rank) * half;
+        const int b_row = x.e * p.C + g.row0 + static_cast<int>(rank) * g.half;
         if (x.kind == 2) {
           // every GEMM-1 tile of this chunk must have stored its slice of H
           const unsigned int need = static_cast<unsigned int>(kCtrPerTile * p.nm1);
           if (!wait_count(p.chunk_ctr + x.e * p.maxc + x.c, need, ab)) break;
           fence_proxy_async_global();  // generic-proxy H stores -> async-proxy (TMA) reads
         }
-        // the token half is one box of the smallest of 128/64/32/16/8 rows that
-        // holds it: one TMA per operand and stage (rows past the chunk load
-        // but no MMA reads them)
+        // the CTA's token rows are one box of the smallest of 256/128/.../8
+        // rows that holds them: one TMA per operand and stage (rows past the
+        // chunk load but no MMA reads them)
         int box = 0;
-        while (box + 1 < kBoxes && (kHalf >> (box + 1)) >= half) ++box;
-        const uint32_t tx = static_cast<uint32_t>(2 * (kABytes + (kHalf >> box) * kBK * 2));
+        while (box + 1 < kBoxes && (kBRowsMax >> (box + 1)) >= g.half) ++box;
+        const uint32_t tx = static_cast<uint32_t>(2 * (kABytes + (kBRowsMax >> box) * kBK * 2));
         bool ok = true;
         for (int kb = 0; kb < K / kBK; ++kb) {
           if (!dev::mbar_wait(&empty_bar[stage], phase ^ 1u, ab)) { ok = false; break; }
@@ -500,14 +541,12 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
         if (++slot == kRing) { slot = 0; rphase ^= 1u; }
         if (t < 0) break;
         const Tile x = sc.decode(t);
-        const int base = s_base[x.e];
-        const int rows_c = min(base, s_rows[x.e] - x.c * base);
-        const int N = (rows_c + kNStep - 1) / kNStep * kNStep;
-        const uint32_t idesc = dev::idesc_bf16_f32(kBM, N);
+        const Geo g = chunk_geo(s_rows[x.e], x.c);
+        const uint32_t idesc = dev::idesc_bf16_f32(kBM, g.N);
         const int num_kb = (x.kind == 1 ? p.d : p.f) / kBK;
         if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, ab)) break;
         dev::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kMaxN);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!dev::mbar_wait(&full_bar[stage], phase, ab)) { ok = false; break; }
@@ -532,8 +571,9 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5 of both CTAs ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    // ---------------- epilogue: warps 2..9 of both CTAs ----------------
+    const int q = warp & 3;          // TMEM lane quarter this warp may read
+    const int hsel = (warp - 2) >> 2;  // which alternate 32-column blocks it stores
     const uint32_t tempty_c0 = mapa(&tempty_bar[0], 0);
     const uint32_t tempty_c1 = mapa(&tempty_bar[1], 0);
     int slot = 0;
@@ -559,84 +599,57 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       dev::tc_fence_after();
-      const int base = s_base[x.e];
-      const int row0 = x.c * base;
-      const int rows_c = min(base, s_rows[x.e] - row0);
-      const int N = (rows_c + kNStep - 1) / kNStep * kNStep;
+      const Geo g = chunk_geo(s_rows[x.e], x.c);
       const int feat = x.m * kBM + static_cast<int>(rank) * kHalf + q * 32 + lane;  // this lane's
-      const int64_t row_base = static_cast<int64_t>(x.e) * p.C + row0;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * kAccStride);
-      if (x.kind == 1) {
-        const int fe = feat & ~1;
-        if (p.glu) {
-          const int unit_even = (feat >> 2) << 1;
-          const bool unit_ok = feat < p.n1;
-#pragma unroll 1
-          for (int n0 = 0; n0 < N; n0 += 32) {
-            uint32_t r[32];
-            if (N - n0 >= 32) {
-              dev::tmem_ld_32x32b_x32(tbase + n0, r);
-              dev::tmem_wait_ld();
-              store_geglu<32>(r, lane, n0, rows_c, p.H, row_base, p.f, unit_even, unit_ok);
-            } else {
-              uint32_t r16[16];
-              dev::tmem_ld_32x32b_x16(tbase + n0, r16);
-              dev::tmem_wait_ld();
+      const int64_t row_base = static_cast<int64_t>(x.e) * p.C + g.row0;
+      for (int n0 = 32 * hsel; n0 < g.N; n0 += 64) {
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * kMaxN + n0);
+        uint32_t r[32];
+        const bool full = g.N - n0 >= 32;
+        if (full) {
+          dev::tmem_ld_32x32b_x32(taddr, r);
+        } else {
+          uint32_t r16[16];
+          dev::tmem_ld_32x32b_x16(taddr, r16);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) r[i] = r16[i];
-              store_geglu<16>(r, lane, n0, rows_c, p.H, row_base, p.f, unit_even, unit_ok);
-            }
+          for (int i = 0; i < 16; ++i) r[i] = r16[i];
+        }
+        dev::tmem_wait_ld();
+        if (x.kind == 1) {
+          if (p.glu) {
+            const int unit_even = (feat >> 2) << 1;
+            const bool unit_ok = feat < p.n1;
+            if (full) store_geglu<32>(r, lane, g, n0, p.H, row_base, p.f, unit_even, unit_ok);
+            else store_geglu<16>(r, lane, g, n0, p.H, row_base, p.f, unit_even, unit_ok);
+          } else {
+            const int fe = feat & ~1;
+            const bool fe_ok = fe < p.n1;
+            if (full)
+              store_pairs<32, true, false>(r, lane, g, n0, p.H, row_base, p.f, fe, fe_ok, 0, 1.f);
+            else
+              store_pairs<16, true, false>(r, lane, g, n0, p.H, row_base, p.f, fe, fe_ok, 0, 1.f);
           }
         } else {
-          const bool fe_ok = fe < p.n1;
-#pragma unroll 1
-          for (int n0 = 0; n0 < N; n0 += 32) {
-            uint32_t r[32];
-            if (N - n0 >= 32) {
-              dev::tmem_ld_32x32b_x32(tbase + n0, r);
-              dev::tmem_wait_ld();
-              store_pairs<32, true, false>(r, lane, n0, rows_c, p.H, row_base, p.f, fe, fe_ok, 0, 1.f);
-            } else {
-              uint32_t r16[16];
-              dev::tmem_ld_32x32b_x16(tbase + n0, r16);
-              dev::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) r[i] = r16[i];
-              store_pairs<16, true, false>(r, lane, n0, rows_c, p.H, row_base, p.f, fe, fe_ok, 0, 1.f);
+          const int fe = feat & ~1;
+          const bool fe_ok = fe < p.d;
+          if (p.y) {
+            // top-1 combine: y[t] = gate_t * E(x_t), into token order
+            int tok_lane = 0;
+            float g_lane = 1.f;
+            if (n0 + lane < g.rows) {
+              tok_lane = __ldg(p.tok_of_row + row_base + n0 + lane);
+              g_lane = __ldg(p.gate + tok_lane);
             }
-          }
-        }
-      } else {
-        const int fe = feat & ~1;
-        const bool fe_ok = fe < p.d;
-        const bool scatter = p.y != nullptr;
-#pragma unroll 1
-        for (int n0 = 0; n0 < N; n0 += 32) {
-          int tok_lane = 0;
-          float g_lane = 1.f;
-          if (scatter && n0 + lane < rows_c) {
-            tok_lane = __ldg(p.tok_of_row + row_base + n0 + lane);
-            g_lane = __ldg(p.gate + tok_lane);
-          }
-          uint32_t r[32];
-          if (N - n0 >= 32) {
-            dev::tmem_ld_32x32b_x32(tbase + n0, r);
-            dev::tmem_wait_ld();
-            if (scatter)
-              store_pairs<32, false, true>(r, lane, n0, rows_c, p.y, 0, p.d, fe, fe_ok, tok_lane, g_lane);
+            if (full)
+              store_pairs<32, false, true>(r, lane, g, n0, p.y, 0, p.d, fe, fe_ok, tok_lane, g_lane);
             else
-              store_pairs<32, false, false>(r, lane, n0, rows_c, p.ye, row_base, p.d, fe, fe_ok, 0, 1.f);
+              store_pairs<16, false, true>(r, lane, g, n0, p.y, 0, p.d, fe, fe_ok, tok_lane, g_lane);
           } else {
-            uint32_t r16[16];
-            dev::tmem_ld_32x32b_x16(tbase + n0, r16);
-            dev::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = r16[i];
-            if (scatter)
-              store_pairs<16, false, true>(r, lane, n0, rows_c, p.y, 0, p.d, fe, fe_ok, tok_lane, g_lane);
+            if (full)
+              store_pairs<32, false, false>(r, lane, g, n0, p.ye, row_base, p.d, fe, fe_ok, 0, 1.f);
             else
-              store_pairs<16, false, false>(r, lane, n0, rows_c, p.ye, row_base, p.d, fe, fe_ok, 0, 1.f);
+              store_pairs<16, false, false>(r, lane, g, n0, p.ye, row_base, p.d, fe, fe_ok, 0, 1.f);
           }
         }
       }
@@ -644,8 +657,8 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
       mbar_arrive_cluster(acc == 0 ? tempty_c0 : tempty_c1);  // CTA 0's accumulator-free barrier
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       if (x.kind == 1) {
-        // publish this warp's 32 features of H for the chunk: its stores are
-        // fenced, then one release increment per warp (8 per tile)
+        // publish this warp's part of H for the chunk: its stores are fenced,
+        // then one release increment per warp
         fence_proxy_async_global();
         __threadfence();
         __syncwarp();
@@ -703,7 +716,7 @@ int32_t make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 }  // namespace
 
 int ffn_pair_chunks(const moe_config& c) {
-  return std::max(1, (c.capacity + kMaxN - 1) / kMaxN);
+  return std::max(1, (c.capacity + kChunk - 1) / kChunk);
 }
 
 int32_t launch_ffn_pair_fused(const moe_config& c, const void* xe, const void* W1, const void* W2,
@@ -725,9 +738,11 @@ int32_t launch_ffn_pair_fused(const moe_config& c, const void* xe, const void* W
   int32_t rc = make_tmap(&maps.w1, W1, static_cast<uint64_t>(E * n1), static_cast<uint64_t>(d), kHalf);
   if (rc == MOE_OK) rc = make_tmap(&maps.w2, W2, static_cast<uint64_t>(E * d), static_cast<uint64_t>(f), kHalf);
   for (int i = 0; i < kBoxes && rc == MOE_OK; ++i) {
-    rc = make_tmap(&maps.x[i], xe, static_cast<uint64_t>(E * C), static_cast<uint64_t>(d), kHalf >> i);
+    rc = make_tmap(&maps.x[i], xe, static_cast<uint64_t>(E * C), static_cast<uint64_t>(d),
+                   kBRowsMax >> i);
     if (rc == MOE_OK)
-      rc = make_tmap(&maps.h[i], H, static_cast<uint64_t>(E * C), static_cast<uint64_t>(f), kHalf >> i);
+      rc = make_tmap(&maps.h[i], H, static_cast<uint64_t>(E * C), static_cast<uint64_t>(f),
+                     kBRowsMax >> i);
   }
   if (rc != MOE_OK) return rc;
   PairParams p{};
@@ -777,7 +792,7 @@ int32_t launch_ffn_pair_fused(const moe_config& c, const void* xe, const void* W
   // L experts, about three tiles per pair (each pair holds up to three tiles
   // between taking one and finishing its epilogue), so their wait for H is
   // normally over when they are taken; chunks per expert estimated as C / 256
-  const int64_t g1_per_expert = std::max<int64_t>(1, static_cast<int64_t>(p.nm1) * C / kMaxN);
+  const int64_t g1_per_expert = std::max<int64_t>(1, static_cast<int64_t>(p.nm1) * C / kChunk);
   p.lag = static_cast<int>(std::min<int64_t>(
       E, std::max<int64_t>(1, (3 * static_cast<int64_t>(resident) + g1_per_expert - 1) /
                                   g1_per_expert)));

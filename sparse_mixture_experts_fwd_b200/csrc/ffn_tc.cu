@@ -449,11 +449,17 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
   const int64_t E = c.E, C = c.capacity, d = c.d_model, f = c.d_ff;
   if (E == 0 || C == 0) return MOE_OK;
   if (C >= 512) {
-    // Experts with hundreds of rows make the GEMMs tensor-core bound: both
-    // GEMMs on SM pairs in one launch, tokens in 16-row steps on the MMA's N
-    // side so a ragged expert wastes almost no MMA rows.
-    return launch_ffn_pair_fused(c, xe, W1, W2, kept_cnt, H, ye, sync, sync_zeroed, status, s,
-                                 top1);
+    // Experts with hundreds of rows make the GEMMs tensor-core bound; SM
+    // pairs feed each SM a third fewer operand bytes per flop than single
+    // CTAs.  With a long GEMM-1 K (d_model >= 2048) both GEMMs run in one
+    // launch with the tokens on the MMA's N side in 16-row steps (a ragged
+    // expert wastes almost no MMA rows, H stays in L2); with a short one the
+    // transposed epilogue of that kernel costs more than it saves, and two
+    // launches with the tokens as M (256-row blocks) measured faster.
+    if (d >= 2048)
+      return launch_ffn_pair_fused(c, xe, W1, W2, kept_cnt, H, ye, sync, sync_zeroed, status,
+                                   s, top1);
+    return launch_ffn_pairs(c, xe, W1, W2, kept_cnt, H, ye, status, s, top1);
   }
   if (C > kBM) {
     // Experts span several 128-row blocks: several CTAs share each weight

@@ -13,7 +13,7 @@ import synth
 @pytest.mark.parametrize("name,C,launches", [
     ("tiny_switch", 32, 3 + 1 + 2 + 1),    # fp32 router, top-k, assign; dispatch; 2 FMA GEMMs; combine
     ("switch_base", 80, 2 + 1 + 1 + 0),    # fused router+top-1, assign; dispatch; fused FFN+combine
-    ("xmoe_top2", 512, 2 + 1 + 1 + 1),     # both GEMMs on SM pairs in one kernel; top-2 combine
+    ("xmoe_top2", 512, 2 + 1 + 2 + 1),     # SM-pair GEMMs (d_model < 2048: two launches); combine
     ("pangu_rre", 640, 2 + 1 + 1 + 0),     # RRE choice, assign; gate 1, combine inside GEMM 2
     ("skewed_switch", 256, 2 + 1 + 2 + 0),
 ])

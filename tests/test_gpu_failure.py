@@ -32,11 +32,11 @@ def moe(cuda_device):
 
 
 # C <= 128: the single-CTA persistent kernel (one counter per expert);
-# C >= 512: the SM-pair kernel (one counter per chunk of at most 256 rows of an
-# expert; expert 0's first chunk is word 1 as well)
+# C >= 512, d >= 2048: the one-launch SM-pair kernel (one counter per chunk of
+# at most 256 rows of an expert; expert 0's first chunk is word 1 as well)
 FFN_CASES = {
     "single_cta": (12, 100, 128, 512, [100, 37, 0, 64, 99, 1, 100, 50, 80, 100, 3, 70]),
-    "sm_pairs": (4, 600, 128, 256, [600, 300, 17, 512]),
+    "sm_pairs": (4, 600, 2048, 256, [600, 300, 17, 512]),
 }
 
 

@@ -203,9 +203,13 @@ FFN_SHAPES = {
     "sm_pairs_long_k": (3, 600, 512, 2048, [600, 0, 513]),
     # C > 512: last 256-row blocks holding 188, 100 (the only block), 128 and 89 rows
     "sm_pairs_tails": (5, 700, 256, 512, [700, 100, 0, 640, 601]),
-    # C >= 512, token chunks of every size class (1, 15, 16, 17 ... 513 rows), feature
+    # C >= 512, experts of every size class (1, 15, 16, 17 ... 513 rows), feature
     # blocks cut short in both GEMMs (d = 192, f = 320)
     "sm_pairs_chunks": (10, 600, 192, 320, [1, 15, 16, 17, 255, 256, 257, 511, 513, 600]),
+    # C >= 512 and d >= 2048: both GEMMs in one SM-pair kernel, tokens on the MMA's N side
+    "sm_pairs_fused": (4, 600, 2048, 256, [600, 1, 513, 256]),
+    # the same kernel: token chunks of every size class, GEMM-1 feature blocks cut short
+    "sm_pairs_fused_chunks": (6, 560, 2048, 320, [1, 17, 255, 257, 513, 560]),
     # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
     "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
 }
