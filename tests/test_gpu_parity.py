@@ -260,7 +260,7 @@ def test_expert_ffn_geglu(moe, cuda_device, shape):
     kept = torch.tensor(kept_list, dtype=torch.int32)
     dt = torch.bfloat16
     xe = synth.normal(22, 1, (E, C, d), 1.0, dt)
-    W1 = synth.normal(22, 3, (E, 2 * f, d), 0.1, dt)
+    W1 = synth.normal(22, 3, (E, 2 * f, d), 0.1 * min(1.0, (512 / d) ** 0.5), dt)  # gate, linear ~N(0, 5) at any d
     W2 = synth.normal(22, 4, (E, d, f), 0.05, dt)
     cfg = moe.make_config(1, d, f, E, 1, C, dtype=dt, expert="geglu")
     H = torch.full((E, C, f), float("nan"), dtype=dt, device=dev)
