@@ -158,7 +158,8 @@ int32_t moe_capacity(int64_t T, int32_t E, double capacity_factor);
 /* MOE_OK if `cfg` is a layer this build runs, else the error code. */
 int32_t moe_config_check(const moe_config* cfg);
 
-/* Bytes of scratch moe_topk_assign needs (0 if cfg is invalid). */
+/* Bytes of scratch moe_topk_assign needs (0 if cfg is invalid).  This build's
+ * assignment exchanges its counts on chip and needs none: 0 for every cfg. */
 size_t moe_assign_workspace_size(const moe_config* cfg);
 
 /* Bytes of scratch moe_expert_ffn needs (0 if cfg is invalid). */
@@ -198,7 +199,8 @@ int32_t moe_router(const moe_config* cfg, const void* x, const void* Wr, const f
  *   n_dropped[0] = sum_e max(0, arrivals[e] - C).
  * Outputs: expert_idx, slot [T, k] int32; gate [T, k] fp32; kept [T, k]
  * uint8; tok_of_row [E*C] int32; arrivals, kept_cnt [E] int32; n_dropped
- * [1] int32.  workspace: moe_assign_workspace_size(cfg) bytes. */
+ * [1] int32.  workspace: moe_assign_workspace_size(cfg) bytes (may be null
+ * when that is 0). */
 int32_t moe_topk_assign(const moe_config* cfg, const float* logits, const int32_t* domain_id,
                         int32_t* expert_idx, float* gate, int32_t* slot, uint8_t* kept,
                         int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,

@@ -182,7 +182,7 @@ int32_t moe_config_check(const moe_config* cfg) {
 
 size_t moe_assign_workspace_size(const moe_config* cfg) {
   if (check_cfg(cfg) != MOE_OK) return 0;
-  return std::max<size_t>(256, assign_scratch_bytes(*cfg));
+  return assign_scratch_bytes(*cfg);
 }
 
 int32_t moe_workspace_layout(const moe_config* cfg, moe_workspace_map* out) {
@@ -407,9 +407,7 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, 
   const bool fused_router = c.mode == MOE_ROUTE_TOPK && c.dtype == MOE_DTYPE_BF16 && c.T > 0;
   if (fused_router) {
     // router GEMM with the gate and top-k in its epilogue (no logits round trip)
-    MOE_TRY(launch_router_topk_tc(c, x, Wr, bias, expert_idx, gate,
-                                  static_cast<unsigned int*>(scratch), assign_flag_words(c),
-                                  status, s));
+    MOE_TRY(launch_router_topk_tc(c, x, Wr, bias, expert_idx, gate, status, s));
   } else if (c.mode == MOE_ROUTE_TOPK && c.T > 0) {
     MOE_TRY(launch_router_f32(c, x, Wr, bias, logits, s));
   }

@@ -151,100 +151,20 @@ struct Sched {
   }
 };
 
-// ---- cluster helpers ----
-MOE_DEV uint32_t cta_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-MOE_DEV void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-MOE_DEV uint32_t mapa(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(dev::smem_u32(p)), "r"(rank));
-  return r;
-}
-MOE_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-MOE_DEV void st_cluster_u32(uint32_t cluster_addr, int v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-// try_wait with cluster-scope acquire: data written by the other CTA of the
-// pair before its release-arrive is visible after it
-MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(dev::smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-MOE_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const dev::Abort& ab) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const unsigned long long t0 = dev::globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (ab.raised()) return false;
-      if (dev::globaltimer() - t0 > ab.limit_ns) {
-        ab.raise();
-        return false;
-      }
-    }
-  }
-}
-MOE_DEV void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t mbar_cluster,
-                              int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dev::smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
-MOE_DEV void tmem_alloc2(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   dev::smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
-}
-MOE_DEV void tmem_relinquish2() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-MOE_DEV void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-MOE_DEV void umma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// arrive on the barrier at this shared offset in both CTAs of the pair once
-// every MMA issued so far has completed
-MOE_DEV void umma2_commit_both(const uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(dev::smem_u32(bar)),
-      "h"(static_cast<uint16_t>(0x3))
-      : "memory");
-}
-MOE_DEV void umma2_commit_local(const uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          dev::smem_u32(bar))
-      : "memory");
-}
+// ---- cluster helpers (shared ones in moe_internal.cuh) ----
+using dev::cluster_sync;
+using dev::cta_rank;
+using dev::mapa;
+using dev::mbar_arrive_cluster;
+using dev::mbar_wait_cluster;
+using dev::st_cluster_u32;
+using dev::tma_load_2d_pair;
+using dev::tmem_alloc2;
+using dev::tmem_dealloc2;
+using dev::tmem_relinquish2;
+using dev::umma2_bf16;
+using dev::umma2_commit_both;
+using dev::umma2_commit_local;
 
 MOE_DEV unsigned int ld_acquire_u32(const unsigned int* p) {
   unsigned int v;
@@ -463,7 +383,7 @@ ffn_pair_kernel(const __grid_constant__ Maps maps, PairParams p) {
         run = publish(cur);
         if (cur >= 0) pending = atomicAdd(p.tile_ctr, 1u);
       }
-      while (run && !ab.raised()) {
+      while (run && !ab.raised_here()) {
         int t;
         if (rank == 0) {
           t = cur;

@@ -224,7 +224,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      while (!ab.raised()) {
+      while (!ab.raised_here()) {
         int t = static_cast<int>(atomicAdd(p.tile_ctr, 1u));
         if (t < 0 || t >= total) t = -1;  // (negative only from a counter not zeroed)
         if (!dev::mbar_wait(&ring_empty[slot], rphase ^ 1u, ab)) break;

@@ -5,8 +5,11 @@
 // for every group g (an expert, or the single router group), m < rows[g]
 // (read on the device, e.g. the kept-token count of an expert) and n < N.
 // Both operands are K-major bf16; accumulation is fp32 in tensor memory.
-// It computes the router logits (Switch notes sec. 2.1 h = W_r x, fp32 per
-// sec. 2.4): x Wr^T + bias.  (The expert FFN has its own fused kernel.)
+// It computes the router logits of moe_router (Switch notes sec. 2.1
+// h = W_r x, fp32 per sec. 2.4: x Wr^T + bias) and the expert FFN of layers
+// whose capacity lies between the ranges of the fused FFN kernels (two
+// grouped launches).  The router with the gate and top-k in its epilogue is
+// router_pair.cu.
 //
 // Design: one persistent CTA per SM walks a static list of 128 x BN output
 // tiles ordered (group, n-block, m-block) so that the m-blocks sharing a
@@ -26,11 +29,9 @@
 namespace moe {
 namespace {
 
-// EPI_TOPK: the router's epilogue computes the gate and top-k itself (Switch
-// notes sec. 2.1, eq. 1) from the token's logits in TMEM instead of storing them.
 // EPI_GLU_BF16: GEMM 1 of a GEGLU expert; accumulator columns 2i, 2i + 1 are
 // hidden unit i's gate and linear parts, out gets GELU(gate) * linear.
-enum EpiKind { EPI_RELU_BF16 = 0, EPI_BF16 = 1, EPI_F32_BIAS = 2, EPI_TOPK = 3, EPI_GLU_BF16 = 4 };
+enum EpiKind { EPI_RELU_BF16 = 0, EPI_BF16 = 1, EPI_F32_BIAS = 2, EPI_GLU_BF16 = 4 };
 
 constexpr int kBM = 128;          // rows per tile (MMA M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
@@ -49,12 +50,7 @@ struct GemmParams {
   int32_t K;
   void* out;                   // row-major, out_ld elements per row
   int64_t out_ld;
-  const float* bias;           // EPI_F32_BIAS / EPI_TOPK, nullable
-  int topk;                    // EPI_TOPK: k (1 or 2)
-  int32_t* expert_idx;         // EPI_TOPK: [T, k]
-  float* gate;                 // EPI_TOPK: [T, k]
-  unsigned int* clear;         // nullable: words block 0 zeroes for the next kernel
-  int n_clear;
+  const float* bias;           // EPI_F32_BIAS, nullable
   const int32_t* scatter_tok;  // EPI_BF16, top-1 layers: row -> token map, or null
   const float* scatter_gate;   //   gate per token
   __nv_bfloat16* scatter_y;    //   y [T, out_ld] written instead of out
@@ -109,7 +105,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_rows[kMaxGroups], s_mblk[kMaxGroups], s_prefix[kMaxGroups + 1];
   __shared__ volatile int s_abort;
-  __shared__ float s_bias[EPI == EPI_TOPK ? BN : 1];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -153,10 +148,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     s_rows[g] = r;
     s_mblk[g] = (r + kBM - 1) / kBM;
   }
-  if (p.clear && blockIdx.x == 0)
-    for (int i = tid; i < p.n_clear; i += kThreads) p.clear[i] = 0u;
-  if constexpr (EPI == EPI_TOPK)
-    for (int i = tid; i < BN; i += kThreads) s_bias[i] = (p.bias && i < p.N) ? p.bias[i] : 0.f;
   __syncthreads();
   if (tid == 0) {
     int acc = 0;
@@ -179,7 +170,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = blockIdx.x; t < total_tiles && !ab.raised(); t += gridDim.x) {
+      for (int t = blockIdx.x; t < total_tiles && !ab.raised_here(); t += gridDim.x) {
         TileCoord tc = tile_of(t, s_prefix, s_mblk, G, n_blocks);
         const int a_row = tc.g * p.a_group_rows + tc.m_blk * kBM;
         const int b_row = tc.g * p.b_group_rows + tc.n_blk * BN;
@@ -209,7 +200,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
-      for (int t = blockIdx.x; t < total_tiles && !ab.raised(); t += gridDim.x) {
+      for (int t = blockIdx.x; t < total_tiles && !ab.raised_here(); t += gridDim.x) {
         if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, ab)) break;
         dev::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
@@ -260,83 +251,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int n0 = tc.n_blk * BN;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * C::kAccStride);
-      if constexpr (EPI == EPI_TOPK) {
-        // One thread = one token; its E logits are re-read from TMEM in a few
-        // passes whose per-element work is independent (4 partial results),
-        // so a single warp per sub-partition keeps its pipelines busy:
-        //   pass 1  m  = max_e h_e
-        //   pass 2  i1 = lowest e with h_e == m;  sum = sum_e exp(h_e - m);
-        //           (top-2) ties = #{e : h_e == m}, below = max{h_e : h_e < m}
-        //   pass 3  (top-2) i2 = lowest e != i1 with h_e == m2, where m2 = m
-        //           if the maximum is tied, else `below`
-        // which is the (value desc, index asc) order of the top-k definition.
-        auto chunk = [&](int c, float (&v)[16]) {
-          uint32_t r[16];
-          dev::tmem_ld_32x32b_x16(tbase + c * 16, r);
-          dev::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c * 16 + i;
-            v[i] = e < p.N ? __uint_as_float(r[i]) + s_bias[e] : -INFINITY;
-          }
-        };
-        float v[16];
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int c = 0; c < BN / 16; ++c) {
-          chunk(c, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx[i & 3] = fmaxf(mx[i & 3], v[i]);
-        }
-        const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        const bool two = p.topk == 2;
-        int i1p[4] = {INT_MAX, INT_MAX, INT_MAX, INT_MAX}, tie[4] = {0, 0, 0, 0};
-        float sp[4] = {0.f, 0.f, 0.f, 0.f};
-        float bl[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int c = 0; c < BN / 16; ++c) {
-          chunk(c, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c * 16 + i;
-            const bool eq = v[i] == m;
-            i1p[i & 3] = (eq && e < i1p[i & 3]) ? e : i1p[i & 3];
-            sp[i & 3] += __expf(v[i] - m);
-            if (two) {
-              tie[i & 3] += eq ? 1 : 0;
-              bl[i & 3] = v[i] < m ? fmaxf(bl[i & 3], v[i]) : bl[i & 3];
-            }
-          }
-        }
-        const int i1 = min(min(i1p[0], i1p[1]), min(i1p[2], i1p[3]));
-        const float ssum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
-        int i2 = INT_MAX;
-        float m2 = -INFINITY;
-        if (two) {
-          m2 = (tie[0] + tie[1] + tie[2] + tie[3]) >= 2
-                   ? m : fmaxf(fmaxf(bl[0], bl[1]), fmaxf(bl[2], bl[3]));
-          int i2p[4] = {INT_MAX, INT_MAX, INT_MAX, INT_MAX};
-#pragma unroll 1
-          for (int c = 0; c < BN / 16; ++c) {
-            chunk(c, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int e = c * 16 + i;
-              i2p[i & 3] = (v[i] == m2 && e != i1 && e < i2p[i & 3]) ? e : i2p[i & 3];
-            }
-          }
-          i2 = min(min(i2p[0], i2p[1]), min(i2p[2], i2p[3]));
-        }
-        if (row_ok) {
-          const int kk = p.topk;
-          p.expert_idx[grow * kk] = i1;
-          p.gate[grow * kk] = 1.0f / ssum;  // exp(m - m) / sum
-          if (two) {
-            p.expert_idx[grow * kk + 1] = i2;
-            p.gate[grow * kk + 1] = expf(m2 - m) / ssum;
-          }
-        }
-      } else if constexpr (EPI == EPI_F32_BIAS) {
+      if constexpr (EPI == EPI_F32_BIAS) {
         float* out = static_cast<float*>(p.out) + grow * p.out_ld;
 #pragma unroll 1
         for (int c = 0; c < BN / 16; ++c) {
@@ -540,40 +455,6 @@ int32_t launch_router_tc(const moe_config& c, const void* x, const void* Wr, con
   if (c.E <= 64) return launch_gemm<64, EPI_F32_BIAS>(x, T, Wr, E, p, tiles, s);
   if (c.E <= 128) return launch_gemm<128, EPI_F32_BIAS>(x, T, Wr, E, p, tiles, s);
   return launch_gemm<256, EPI_F32_BIAS>(x, T, Wr, E, p, tiles, s);
-}
-
-// Router with the gate and top-k in its epilogue: expert_idx/gate [T, k]
-// without writing logits.  Block 0 also zeroes `clear` (n_clear words) for
-// the slot-assignment kernel that follows on the stream.
-int32_t launch_router_topk_tc(const moe_config& c, const void* x, const void* Wr,
-                              const float* bias, int32_t* expert_idx, float* gate,
-                              unsigned int* clear, int n_clear, int32_t* status, cudaStream_t s) {
-  if (c.T == 0) return MOE_OK;
-  GemmParams p{};
-  p.num_groups = 1;
-  p.a_group_rows = 0;
-  p.group_rows = nullptr;
-  p.fixed_rows = static_cast<int32_t>(c.T);
-  p.max_rows = static_cast<int32_t>(c.T);
-  p.N = c.E;
-  p.b_group_rows = 0;
-  p.K = c.d_model;
-  p.out = nullptr;
-  p.out_ld = 0;
-  p.bias = bias;
-  p.topk = c.k;
-  p.expert_idx = expert_idx;
-  p.gate = gate;
-  p.clear = clear;
-  p.n_clear = n_clear;
-  p.status = status;
-  p.wait_ns = wait_limit_ns();
-  const int64_t tiles = (c.T + kBM - 1) / kBM;
-  const uint64_t T = static_cast<uint64_t>(c.T), E = static_cast<uint64_t>(c.E);
-  if (c.E <= 32) return launch_gemm<32, EPI_TOPK>(x, T, Wr, E, p, tiles, s);
-  if (c.E <= 64) return launch_gemm<64, EPI_TOPK>(x, T, Wr, E, p, tiles, s);
-  if (c.E <= 128) return launch_gemm<128, EPI_TOPK>(x, T, Wr, E, p, tiles, s);
-  return launch_gemm<256, EPI_TOPK>(x, T, Wr, E, p, tiles, s);
 }
 
 }  // namespace moe

@@ -63,69 +63,16 @@ struct Gemm2Params {
   __nv_bfloat16* scatter_y;    //   y [T, out_ld] written instead of out
 };
 
-MOE_DEV uint32_t cta_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-MOE_DEV void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-// shared::cluster address of `p` (a shared variable) in CTA `rank` of the cluster
-MOE_DEV uint32_t mapa(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(dev::smem_u32(p)), "r"(rank));
-  return r;
-}
-MOE_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-MOE_DEV void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t mbar_cluster,
-                              int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dev::smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
-MOE_DEV void tmem_alloc2(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   dev::smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
-}
-MOE_DEV void tmem_relinquish2() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-MOE_DEV void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-MOE_DEV void umma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
-      : "memory");
-}
-// arrive on the barrier at this shared offset in both CTAs of the pair once
-// every MMA issued so far has completed
-MOE_DEV void umma2_commit_both(const uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(dev::smem_u32(bar)),
-      "h"(static_cast<uint16_t>(0x3))
-      : "memory");
-}
-MOE_DEV void umma2_commit_local(const uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          dev::smem_u32(bar))
-      : "memory");
-}
+using dev::cluster_sync;
+using dev::cta_rank;
+using dev::mapa;
+using dev::mbar_arrive_cluster;
+using dev::tma_load_2d_pair;
+using dev::tmem_alloc2;
+using dev::tmem_dealloc2;
+using dev::tmem_relinquish2;
+using dev::umma2_commit_both;
+using dev::umma2_commit_local;
 
 struct TileCoord {
   int g, m, n;  // m: 256-row block
@@ -219,7 +166,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      for (int t = cluster; t < total && !ab.raised(); t += n_clusters) {
+      for (int t = cluster; t < total && !ab.raised_here(); t += n_clusters) {
         const TileCoord tc = tile_of(t, s_prefix, s_mblk, G);
         const int a_row = tc.g * p.a_group_rows + tc.m * kBM + static_cast<int>(rank) * kHalf;
         const int b_row = tc.g * p.b_group_rows + tc.n * kBN + static_cast<int>(rank) * kHalf;
@@ -252,7 +199,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
-      for (int t = cluster; t < total && !ab.raised(); t += n_clusters) {
+      for (int t = cluster; t < total && !ab.raised_here(); t += n_clusters) {
         if (!dev::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, ab)) break;
         dev::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccStride);
@@ -264,7 +211,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint64_t bdesc = dev::smem_desc_k_sw128(dev::smem_u32(smB + stage * kBBytes));
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk)
-            umma2_bf16(d_tmem, adesc + 2ull * kk, bdesc + 2ull * kk, (kb > 0 || kk > 0) ? 1u : 0u);
+            dev::umma2_bf16(d_tmem, adesc + 2ull * kk, bdesc + 2ull * kk, kIdesc,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
           umma2_commit_both(&empty_bar[stage]);
           any = true;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }

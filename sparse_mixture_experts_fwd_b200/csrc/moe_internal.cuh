@@ -102,12 +102,9 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
                             int32_t* n_dropped, void* scratch, int32_t* status,
                             cudaStream_t s);
 size_t assign_scratch_bytes(const moe_config& c);
-// look-back flags at the start of the assignment scratch; the kernel that
-// produces the choices zeroes them
-int assign_flag_words(const moe_config& c);
 int32_t launch_router_topk_tc(const moe_config& c, const void* x, const void* Wr,
                               const float* bias, int32_t* expert_idx, float* gate,
-                              unsigned int* clear, int n_clear, int32_t* status, cudaStream_t s);
+                              int32_t* status, cudaStream_t s);
 int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* slot,
                       uint8_t* kept, int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
                       int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s);
@@ -172,6 +169,10 @@ struct Abort {
     if (*local) return true;
     return status && (*reinterpret_cast<volatile int32_t*>(status) & MOE_STATUS_TIMEOUT);
   }
+  // The CTA's own flag only: a shared-memory read, for the per-tile checks of
+  // producer and MMA loops (the status word is a global-memory round trip;
+  // the bounded waits poll it)
+  MOE_DEV bool raised_here() const { return *local != 0; }
   MOE_DEV void raise() const {
     *local = 1;
     if (status) atomicOr(status, MOE_STATUS_TIMEOUT);
@@ -318,6 +319,104 @@ MOE_DEV void umma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+// -- SM pairs (thread-block clusters of two CTAs, tcgen05 cta_group::2) --
+MOE_DEV uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+MOE_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// shared::cluster address of `p` (a shared variable) in CTA `rank` of the cluster
+MOE_DEV uint32_t mapa(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+MOE_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+MOE_DEV void st_cluster_u32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// try_wait with cluster-scope acquire: data written by the other CTA of the
+// pair before its release-arrive is visible after it
+MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+MOE_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (ab.raised()) return false;
+      if (globaltimer() - t0 > ab.limit_ns) {
+        ab.raise();
+        return false;
+      }
+    }
+  }
+}
+// TMA load into this CTA's shared memory whose completion is counted on the
+// barrier `mbar_cluster` (a shared::cluster address, normally CTA 0's)
+MOE_DEV void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t mbar_cluster,
+                              int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+MOE_DEV void tmem_alloc2(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+MOE_DEV void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+MOE_DEV void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+MOE_DEV void umma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this shared offset in both CTAs of the pair once
+// every MMA issued so far has completed
+MOE_DEV void umma2_commit_both(const uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(0x3))
+      : "memory");
+}
+MOE_DEV void umma2_commit_local(const uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 MOE_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 columns of 32-bit: thread i of the warp gets row (lane base + i),

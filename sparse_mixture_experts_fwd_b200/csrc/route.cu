@@ -7,30 +7,34 @@
 // the same way with the first excluded, and the softmax denominator
 // sum_j exp(h_j - max) with a shuffle sum; gate = exp(h_i - max) / sum.
 //
-// Slot assignment (sec. 2.2, eq. 3 and the drop rule), in token order, as ONE
-// kernel over blocks of 1024 choices (choice a = t*k + j):
-//   1. rank inside the block: __match_any_sync groups the lanes that chose
-//      the same expert, __popc of the lower peers gives the rank inside the
-//      warp, per-warp counts are prefix-summed in shared memory across the 32
-//      warps; the block's per-expert counts are its aggregate;
-//   2. decoupled look-back: the block publishes its aggregate (flag 1), reads
-//      the flags of all earlier blocks, and sums their aggregates back to the
-//      nearest block that already published its inclusive prefix (flag 2),
-//      then publishes its own inclusive prefix (flag 2);
-//   3. slot = exclusive prefix + rank, kept = slot < C, row -> token map;
-//      the last block also writes arrivals, kept counts, the dropped total
-//      and marks free rows of the map with -1.
-// The flags are cleared by the kernel that produced the choices (stream
-// order), and every wait on a flag is bounded by time.
+// Slot assignment (sec. 2.2, eq. 3 and the drop rule), in choice order
+// (choice a = t*k + j), as ONE kernel on ONE thread-block cluster (16 CTAs
+// where the device can co-schedule them, else 8) of 1024 threads each.  The
+// cluster's CTAs are resident together by construction, so they exchange
+// counts through distributed shared memory with the hardware cluster barrier
+// and nothing spins on global flags:
+//   1. each warp owns a contiguous run of choices and counts them per expert
+//      (__match_any_sync groups the lanes that chose the same expert);
+//   2. the 32 warps' counts are prefix-summed per expert in shared memory,
+//      giving the CTA's per-expert total; cluster barrier;
+//   3. each CTA reads every CTA's totals (DSMEM): the sum over earlier CTAs
+//      is its exclusive prefix, the sum over all the arrivals; barrier;
+//   4. each warp walks its run again: slot = earlier CTAs + earlier warps +
+//      earlier rounds of this warp + rank among this round's peers;
+//      kept = slot < C, and the row -> token map;
+//   5. CTA 0 writes arrivals, kept counts and the dropped total; every CTA
+//      marks the free rows of its share of experts with -1.
+#include <algorithm>
 #include <climits>
 #include <cmath>
+#include <mutex>
 
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kAssignBlock = 1024;
+constexpr int kAssignThreads = 1024;
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t t) {
   // output #t of splitmix64 seeded with `seed` (Steele, Lea & Flood 2014)
@@ -38,11 +42,6 @@ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t t) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
   return z ^ (z >> 31);
-}
-
-__device__ __forceinline__ void clear_flags(unsigned int* flags, int nblk) {
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < nblk; i += blockDim.x) flags[i] = 0u;
 }
 
 // logits[t, e] = sum_c x[t, c] * Wr[e, c] + bias[e]   (fp32 FMA chain in c order)
@@ -80,11 +79,9 @@ template <int K>
 __global__ void __launch_bounds__(256) gate_topk_kernel(int64_t T, int E,
                                                         const float* __restrict__ logits,
                                                         int32_t* __restrict__ expert_idx,
-                                                        float* __restrict__ gate,
-                                                        unsigned int* flags, int nblk) {
+                                                        float* __restrict__ gate) {
   dev::pdl_trigger();
   dev::pdl_wait();
-  clear_flags(flags, nblk);
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; t < T;
@@ -137,10 +134,9 @@ __global__ void __launch_bounds__(256) gate_topk_kernel(int64_t T, int E,
 __global__ void route_rre_kernel(int64_t T, int E, int G, uint64_t seed,
                                  const int32_t* __restrict__ domain,
                                  int32_t* __restrict__ expert_idx, float* __restrict__ gate,
-                                 int32_t* status, unsigned int* flags, int nblk) {
+                                 int32_t* status) {
   dev::pdl_trigger();
   dev::pdl_wait();
-  clear_flags(flags, nblk);
   const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (t >= T) return;
   const int per = E / G;
@@ -154,18 +150,16 @@ __global__ void route_rre_kernel(int64_t T, int E, int G, uint64_t seed,
   gate[t] = 1.0f;
 }
 
-MOE_DEV unsigned int ld_acquire(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+MOE_DEV int ld_cluster_s32(uint32_t cluster_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
   return v;
-}
-MOE_DEV void st_release(unsigned int* p, unsigned int v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 struct AssignArgs {
   int64_t n_assign;
-  int k, E, C, nblk;
+  int64_t per_warp;  // choices per warp, a multiple of 32
+  int k, E, C;
   const int32_t* expert_idx;
   int32_t* slot;
   uint8_t* kept;
@@ -173,135 +167,95 @@ struct AssignArgs {
   int32_t* arrivals;
   int32_t* kept_cnt;
   int32_t* n_dropped;
-  unsigned int* flags;  // [nblk], cleared before launch
-  int32_t* aggr;        // [nblk][E]
-  int32_t* incl;        // [nblk][E]
-  int32_t* status;      // nullable; also the call's give-up signal
-  uint64_t wait_ns;     // limit of the look-back wait
 };
 
-__global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArgs p) {
-  extern __shared__ int s_cnt[];  // [32 warps][E], then excl[E]
-  __shared__ int s_pstar, s_ok, s_maxinc, s_maxbad, s_drop[32], s_ticket;
-  int* s_excl = s_cnt + 32 * p.E;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignArgs p) {
+  extern __shared__ int s_mem[];
   const int E = p.E;
+  int* s_cnt = s_mem;           // [32 warps][E]: counts, then bases for the warp's next round
+  int* s_tot = s_cnt + 32 * E;  // [E] this CTA's choices per expert
+  int* s_excl = s_tot + E;      // [E] earlier CTAs' choices per expert
+  int* s_all = s_excl + E;      // [E] all choices per expert (arrivals)
+  __shared__ int s_drop[kAssignThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = static_cast<int>(dev::cta_rank());
+  const int nb = static_cast<int>(gridDim.x);  // the grid is one cluster
+  const int64_t w0 = (static_cast<int64_t>(b) * (kAssignThreads / 32) + warp) * p.per_warp;
+  const int64_t w1 = w0 + p.per_warp < p.n_assign ? w0 + p.per_warp : p.n_assign;
+  const unsigned lower = (1u << lane) - 1u;
 
-  // 1. ranks inside the block
   dev::pdl_trigger();
-  for (int i = tid; i < 32 * E; i += kAssignBlock) s_cnt[i] = 0;
-  dev::pdl_wait();
-  // The block's place in token order is a ticket taken when it starts, not
-  // blockIdx: a block then only ever waits on blocks that are already running,
-  // whatever order the hardware starts them in.
-  if (tid == 0) s_ticket = static_cast<int>(atomicAdd(p.flags + p.nblk, 1u));
+  for (int i = tid; i < 32 * E; i += kAssignThreads) s_cnt[i] = 0;
+  dev::pdl_wait();  // the choices come from the previous kernel
   __syncthreads();
-  const int b = s_ticket;
-  const int64_t a = static_cast<int64_t>(b) * kAssignBlock + tid;
-  int e = a < p.n_assign ? __ldg(p.expert_idx + a) : -1;
-  if (e >= E) e = -1;
-  const unsigned peers = __match_any_sync(0xffffffffu, e);
-  const int r_in_warp = __popc(peers & ((1u << lane) - 1u));
-  if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * E + e] = __popc(peers);
+
+  // 1. this warp's counts per expert (the leader of each group of peers adds)
+#pragma unroll 4
+  for (int64_t base = w0; base < w1; base += 32) {
+    const int64_t a = base + lane;
+    int e = a < w1 ? __ldg(p.expert_idx + a) : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * E + e] += __popc(peers);
+    __syncwarp();  // the next round's leader may be another lane
+  }
   __syncthreads();
-  for (int x = tid; x < E; x += kAssignBlock) {
+  // 2. exclusive prefix over the warps (choice order), CTA totals
+  for (int x = tid; x < E; x += kAssignThreads) {
     int run = 0;
     for (int w = 0; w < 32; ++w) {
       const int c = s_cnt[w * E + x];
       s_cnt[w * E + x] = run;
       run += c;
     }
-    p.aggr[static_cast<int64_t>(b) * E + x] = run;  // block aggregate
-    s_excl[x] = 0;
-    if (b == 0) p.incl[x] = run;
+    s_tot[x] = run;
   }
-  // 2. publish the aggregate (or, for block 0, the inclusive prefix)
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) st_release(p.flags + b, b == 0 ? 2u : 1u);
-
-  if (b > 0) {
-    // p*: the latest earlier block with an inclusive prefix, usable once every
-    // block after it has at least published its aggregate.  All earlier flags
-    // are read in parallel (one thread each) and reduced in shared memory.
-    const unsigned long long t0 = dev::globaltimer();
-    for (;;) {
-      if (tid == 0) {
-        s_maxinc = -1;
-        s_maxbad = -1;
-      }
-      __syncthreads();
-      for (int q = tid; q < b; q += kAssignBlock) {
-        const unsigned int f = ld_acquire(p.flags + q);
-        if (f == 2u) atomicMax(&s_maxinc, q);
-        else if (f == 0u) atomicMax(&s_maxbad, q);
-      }
-      __syncthreads();
-      const bool ready = s_maxinc >= 0 && s_maxbad < s_maxinc;
-      if (tid == 0) {
-        s_pstar = s_maxinc;
-        if (ready) {
-          s_ok = 1;
-        } else if (p.status &&
-                   (*reinterpret_cast<volatile int32_t*>(p.status) & MOE_STATUS_TIMEOUT)) {
-          s_ok = -1;  // another wait of this call has already given up
-        } else if (dev::globaltimer() - t0 > p.wait_ns) {
-          s_ok = -1;
-          if (p.status) atomicOr(p.status, MOE_STATUS_TIMEOUT);
-        } else {
-          s_ok = 0;
-        }
-      }
-      __syncthreads();
-      if (s_ok != 0) break;
+  dev::cluster_sync();  // every CTA's totals are final and visible in the cluster
+  // 3. earlier CTAs' totals (the exclusive prefix) and all CTAs' (the arrivals)
+  for (int x = tid; x < E; x += kAssignThreads) {
+    int before = 0, all = 0;
+    const uint32_t addr = dev::smem_u32(s_tot + x);
+    for (int q = 0; q < nb; ++q) {
+      uint32_t remote;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(q));
+      const int v = ld_cluster_s32(remote);
+      before += q < b ? v : 0;
+      all += v;
     }
-    if (s_ok < 0) return;  // bounded wait expired: outputs are invalid, status says so
-    const int pstar = s_pstar;
-    for (int x = tid; x < E; x += kAssignBlock) {
-      // the aggregates after p* are independent loads: 8 in flight per round
-      int acc = __ldcg(p.incl + static_cast<int64_t>(pstar) * E + x);
-      int part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      int q = pstar + 1;
-      for (; q + 8 <= b; q += 8) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) part[u] += __ldcg(p.aggr + static_cast<int64_t>(q + u) * E + x);
-      }
-      for (; q < b; ++q) part[0] += __ldcg(p.aggr + static_cast<int64_t>(q) * E + x);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc += part[u];
-      s_excl[x] = acc;
-      p.incl[static_cast<int64_t>(b) * E + x] = acc + p.aggr[static_cast<int64_t>(b) * E + x];
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) st_release(p.flags + b, 2u);
-  } else {
-    __syncthreads();
+    s_excl[x] = before;
+    s_all[x] = all;
   }
+  dev::cluster_sync();  // no CTA reads another's shared memory after this (it may exit)
 
-  // 3. slots, kept mask, row -> token map
-  if (a < p.n_assign) {
-    if (e >= 0) {
-      const int s = s_excl[e] + s_cnt[warp * E + e] + r_in_warp;
-      p.slot[a] = s;
-      const bool kp = s < p.C;
+  // 4. slots in choice order
+#pragma unroll 4
+  for (int64_t base = w0; base < w1; base += 32) {
+    const int64_t a = base + lane;
+    const bool in = a < w1;
+    int e = in ? __ldg(p.expert_idx + a) : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int s = INT_MAX;
+    if (e >= 0) s = s_excl[e] + s_cnt[warp * E + e] + __popc(peers & lower);
+    __syncwarp();  // every peer has read the base before the leader moves it
+    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * E + e] += __popc(peers);
+    __syncwarp();
+    if (in) {
+      p.slot[a] = s;  // INT_MAX for an expert index outside [0, E)
+      const bool kp = e >= 0 && s < p.C;
       p.kept[a] = kp ? 1 : 0;
       if (kp) p.tok_of_row[static_cast<int64_t>(e) * p.C + s] = static_cast<int32_t>(a / p.k);
-    } else {
-      p.slot[a] = INT_MAX;
-      p.kept[a] = 0;
     }
   }
-  // the last block owns the totals
-  if (b == p.nblk - 1) {
-    __syncthreads();  // every thread is done reading the rank table reused below
+
+  // 5. totals (CTA 0) and the free rows of the map (experts x = b mod nb, a warp each)
+  if (b == 0) {
     int drop = 0;
-    for (int x = tid; x < E; x += kAssignBlock) {
-      const int arr = s_excl[x] + p.aggr[static_cast<int64_t>(b) * E + x];
-      p.arrivals[x] = arr;
+    for (int x = tid; x < E; x += kAssignThreads) {
+      const int arr = s_all[x];
       const int kc = arr < p.C ? arr : p.C;
+      p.arrivals[x] = arr;
       p.kept_cnt[x] = kc;
-      s_cnt[x] = kc;  // reuse: kept count per expert for the -1 fill below
       drop += arr - kc;
     }
 #pragma unroll
@@ -310,13 +264,14 @@ __global__ void __launch_bounds__(kAssignBlock, 1) assign_kernel(const AssignArg
     __syncthreads();
     if (tid == 0) {
       int tot = 0;
-      for (int w = 0; w < 32; ++w) tot += s_drop[w];
+      for (int w = 0; w < kAssignThreads / 32; ++w) tot += s_drop[w];
       p.n_dropped[0] = tot;
     }
-    // free rows of the map: a warp per expert, lanes over its rows past the kept count
-    for (int ex = warp; ex < E; ex += kAssignBlock / 32)
-      for (int r = s_cnt[ex] + lane; r < p.C; r += 32)
-        p.tok_of_row[static_cast<int64_t>(ex) * p.C + r] = -1;
+  }
+  for (int x = b + nb * warp; x < E; x += nb * (kAssignThreads / 32)) {
+    const int kc = s_all[x] < p.C ? s_all[x] : p.C;
+    for (int r = kc + lane; r < p.C; r += 32)
+      p.tok_of_row[static_cast<int64_t>(x) * p.C + r] = -1;
   }
 }
 
@@ -338,17 +293,9 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace
 
-// the look-back flags [nblk] and the block ticket counter after them
-int assign_flag_words(const moe_config& c) {
-  return static_cast<int>(ceil_div(c.T * c.k, kAssignBlock)) + 1;
-}
-
-// flags [nblk] u32 + ticket u32, then aggr and incl [nblk][E] i32 each
-size_t assign_scratch_bytes(const moe_config& c) {
-  const int64_t nblk = ceil_div(c.T * c.k, kAssignBlock);
-  return align256(static_cast<size_t>(nblk + 1) * sizeof(unsigned int)) +
-         2 * align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
-}
+// The assignment needs no global scratch (its CTAs exchange counts in
+// distributed shared memory).
+size_t assign_scratch_bytes(const moe_config&) { return 0; }
 
 int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, const float* bias,
                           float* logits, cudaStream_t s) {
@@ -365,61 +312,98 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
                             int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
                             int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s) {
   const int64_t T = c.T;
-  const int64_t n_assign = T * c.k;
-  const int64_t nblk = ceil_div(n_assign, kAssignBlock);
-  char* sc = static_cast<char*>(scratch);
-  unsigned int* flags = reinterpret_cast<unsigned int*>(sc);
-  const size_t flags_bytes = align256(static_cast<size_t>(nblk + 1) * sizeof(unsigned int));
-  const size_t vec_bytes = align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
-  int32_t* aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
-  int32_t* incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
-  if (T == 0) {
-    launch_pdl(assign_empty_kernel, dim3(1), dim3(256), 0, s, c.E, c.capacity, arrivals, kept_cnt, n_dropped,
-                                          tok_of_row);
-    return check_launch("assign_empty_kernel");
-  }
-  if (c.mode == MOE_ROUTE_TOPK) {
-    const int64_t blocks = std::min<int64_t>(ceil_div(T, 8), int64_t(num_sms()) * 16);
-    if (c.k == 1)
-      launch_pdl(gate_topk_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
-                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk + 1));
-    else
-      launch_pdl(gate_topk_kernel<2>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
-                 c.E, logits, expert_idx, gate, flags, static_cast<int>(nblk + 1));
-    int32_t rc = check_launch("gate_topk_kernel");
-    if (rc != MOE_OK) return rc;
-  } else {
-    launch_pdl(route_rre_kernel, dim3(static_cast<unsigned>(ceil_div(T, 256))), dim3(256), 0, s,
-               T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status, flags,
-               static_cast<int>(nblk + 1));
-    int32_t rc = check_launch("route_rre_kernel");
-    if (rc != MOE_OK) return rc;
+  if (T > 0) {
+    if (c.mode == MOE_ROUTE_TOPK) {
+      const int64_t blocks = std::min<int64_t>(ceil_div(T, 8), int64_t(num_sms()) * 16);
+      if (c.k == 1)
+        launch_pdl(gate_topk_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
+                   c.E, logits, expert_idx, gate);
+      else
+        launch_pdl(gate_topk_kernel<2>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, T,
+                   c.E, logits, expert_idx, gate);
+      int32_t rc = check_launch("gate_topk_kernel");
+      if (rc != MOE_OK) return rc;
+    } else {
+      launch_pdl(route_rre_kernel, dim3(static_cast<unsigned>(ceil_div(T, 256))), dim3(256), 0, s,
+                 T, c.E, c.num_groups, c.seed, domain, expert_idx, gate, status);
+      int32_t rc = check_launch("route_rre_kernel");
+      if (rc != MOE_OK) return rc;
+    }
   }
   return launch_assign(c, expert_idx, slot, kept, tok_of_row, arrivals, kept_cnt, n_dropped,
                        scratch, status, s);
 }
 
-// The slot assignment alone, from choices whose look-back flags are already
-// cleared (by the kernel that produced them, earlier on the same stream).
+namespace {
+
+size_t assign_smem_bytes(int E) { return (32 + 3) * static_cast<size_t>(E) * sizeof(int); }
+
+// CTAs in the assignment's cluster: 16 where the device co-schedules a
+// cluster of 16 such CTAs (a non-portable size), else the portable 8.
+// Queried once per device.
+int32_t assign_cluster_size(int* out) {
+  constexpr int kMaxDev = 64;
+  static int cache[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < kMaxDev && cache[dev] > 0) {
+    *out = cache[dev];
+    return MOE_OK;
+  }
+  const size_t smem = assign_smem_bytes(256);
+  if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+    return check_launch("cudaFuncSetAttribute(assign_kernel)");
+  int size = 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(16);
+  cfg.blockDim = dim3(kAssignThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, assign_kernel, &cfg) == cudaSuccess && clusters >= 1)
+    size = 16;
+  cudaGetLastError();  // a refused query leaves no error behind
+  if (dev < kMaxDev) cache[dev] = size;
+  *out = size;
+  return MOE_OK;
+}
+
+}  // namespace
+
+// The slot assignment alone, from the choices expert_idx [T, k] written
+// earlier on the same stream.
 int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* slot,
                       uint8_t* kept, int32_t* tok_of_row, int32_t* arrivals, int32_t* kept_cnt,
                       int32_t* n_dropped, void* scratch, int32_t* status, cudaStream_t s) {
+  (void)scratch;
+  (void)status;
   const int64_t n_assign = c.T * c.k;
-  const int64_t nblk = ceil_div(n_assign, kAssignBlock);
-  if (nblk == 0) {
-    launch_pdl(assign_empty_kernel, dim3(1), dim3(256), 0, s, c.E, c.capacity, arrivals, kept_cnt, n_dropped,
-                                          tok_of_row);
+  if (n_assign == 0) {
+    launch_pdl(assign_empty_kernel, dim3(1), dim3(256), 0, s, c.E, c.capacity, arrivals, kept_cnt,
+               n_dropped, tok_of_row);
     return check_launch("assign_empty_kernel");
   }
-  char* sc = static_cast<char*>(scratch);
-  const size_t flags_bytes = align256(static_cast<size_t>(nblk + 1) * sizeof(unsigned int));
-  const size_t vec_bytes = align256(static_cast<size_t>(nblk) * c.E * sizeof(int32_t));
+  int nb = 0;
+  int32_t rc = assign_cluster_size(&nb);
+  if (rc != MOE_OK) return rc;
   AssignArgs p{};
   p.n_assign = n_assign;
+  // choices per warp: the whole list over nb * 32 warps, in rounds of 32
+  p.per_warp = ceil_div(ceil_div(n_assign, int64_t(nb) * (kAssignThreads / 32)), 32) * 32;
   p.k = c.k;
   p.E = c.E;
   p.C = c.capacity;
-  p.nblk = static_cast<int>(nblk);
   p.expert_idx = expert_idx;
   p.slot = slot;
   p.kept = kept;
@@ -427,13 +411,21 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
   p.arrivals = arrivals;
   p.kept_cnt = kept_cnt;
   p.n_dropped = n_dropped;
-  p.flags = reinterpret_cast<unsigned int*>(sc);
-  p.aggr = reinterpret_cast<int32_t*>(sc + flags_bytes);
-  p.incl = reinterpret_cast<int32_t*>(sc + flags_bytes + vec_bytes);
-  p.status = status;
-  p.wait_ns = wait_limit_ns();
-  const size_t smem = (33 * static_cast<size_t>(c.E)) * sizeof(int);
-  launch_pdl(assign_kernel, dim3(static_cast<unsigned>(nblk)), dim3(kAssignBlock), smem, s, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nb));
+  cfg.blockDim = dim3(kAssignThreads);
+  cfg.dynamicSmemBytes = assign_smem_bytes(c.E);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(nb);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaLaunchKernelEx(&cfg, assign_kernel, p);
   return check_launch("assign_kernel");
 }
 

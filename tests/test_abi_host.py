@@ -101,9 +101,11 @@ def test_calls_rejected_on_host(moe):
     # workspace too small
     assert moe.lib.moe_layer_forward(ctypes.byref(c), p, p, None, None, p, p, p, p, 10, None, None,
                                      None) == -4
-    # topk_assign without workspace
-    assert moe.lib.moe_topk_assign(ctypes.byref(c), p, None, p, p, p, p, p, p, p, p, None, 0,
-                                   None, None) == -4
+    # topk_assign without its gate output
+    assert moe.lib.moe_topk_assign(ctypes.byref(c), p, None, p, None, p, p, p, p, p, p, None, 0,
+                                   None, None) == -1
+    # the assignment takes no scratch: the size is 0 and a null workspace passes validation
+    assert moe.lib.moe_assign_workspace_size(ctypes.byref(c)) == 0
     # invalid config reaches no launch
     bad = cfg(moe, k=3)
     assert moe.lib.moe_expert_ffn(ctypes.byref(bad), p, p, p, p, p, p, p, 4096, None, None) == -2
