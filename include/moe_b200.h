@@ -226,10 +226,12 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* expert
  * rows of H and ye are left untouched.  bf16 runs tcgen05 kernels with fp32
  * accumulation, chosen by the capacity: C <= 128, one persistent kernel for
  * both GEMMs (128 x 256 tiles); 128 < C < 512, two grouped launches (one per
- * GEMM, 128 x 256 tiles); C >= 512, two grouped launches on SM pairs
- * (256 x 256 tiles, cta_group::2).  workspace: moe_ffn_workspace_size bytes
- * (zeroed by the call; the persistent kernel's tile counters).  fp32 runs
- * FMA GEMMs and may pass a null workspace. */
+ * GEMM, 128 x 256 tiles); C >= 512, SM pairs (cta_group::2): with
+ * d_model >= 2048 one persistent kernel for both GEMMs (256 weight rows x up
+ * to 256 tokens per tile), else two grouped launches (256 x 256 tiles).
+ * workspace: moe_ffn_workspace_size bytes (zeroed by the call; the persistent
+ * kernels' tile and dependency counters).  fp32 runs FMA GEMMs and may pass
+ * a null workspace. */
 int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const void* W1, const void* W2,
                        const int32_t* kept_cnt, void* H, void* ye, void* workspace,
                        size_t workspace_bytes, int32_t* status, moe_stream_t stream);

@@ -35,6 +35,7 @@ namespace moe {
 namespace {
 
 constexpr int kAssignThreads = 1024;
+constexpr int kMaxAssignCtas = 16;  // CTAs in the assignment's cluster (16 or 8)
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t t) {
   // output #t of splitmix64 seeded with `seed` (Steele, Lea & Flood 2014)
@@ -172,8 +173,11 @@ struct AssignArgs {
 __global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignArgs p) {
   extern __shared__ int s_mem[];
   const int E = p.E;
-  int* s_cnt = s_mem;           // [32 warps][E]: counts, then bases for the warp's next round
-  int* s_tot = s_cnt + 32 * E;  // [E] this CTA's choices per expert
+  // [32 warps][Ep]: counts, then bases for the warp's next round; the odd
+  // row stride Ep keeps a column (one expert, all warps) in 32 banks
+  const int Ep = E | 1;
+  int* s_cnt = s_mem;
+  int* s_tot = s_cnt + 32 * Ep;  // [E] this CTA's choices per expert
   int* s_excl = s_tot + E;      // [E] earlier CTAs' choices per expert
   int* s_all = s_excl + E;      // [E] all choices per expert (arrivals)
   __shared__ int s_drop[kAssignThreads / 32];
@@ -185,7 +189,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignA
   const unsigned lower = (1u << lane) - 1u;
 
   dev::pdl_trigger();
-  for (int i = tid; i < 32 * E; i += kAssignThreads) s_cnt[i] = 0;
+  for (int i = tid; i < 32 * Ep; i += kAssignThreads) s_cnt[i] = 0;
   dev::pdl_wait();  // the choices come from the previous kernel
   __syncthreads();
 
@@ -196,31 +200,43 @@ __global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignA
     int e = a < w1 ? __ldg(p.expert_idx + a) : -1;
     if (e < 0 || e >= E) e = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * E + e] += __popc(peers);
+    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * Ep + e] += __popc(peers);
     __syncwarp();  // the next round's leader may be another lane
   }
   __syncthreads();
-  // 2. exclusive prefix over the warps (choice order), CTA totals
-  for (int x = tid; x < E; x += kAssignThreads) {
-    int run = 0;
-    for (int w = 0; w < 32; ++w) {
-      const int c = s_cnt[w * E + x];
-      s_cnt[w * E + x] = run;
-      run += c;
+  // 2. exclusive prefix over the warps (choice order), CTA totals: a warp per
+  //    expert, lane w holding warp w's count, scanned with shuffles
+  for (int x = warp; x < E; x += kAssignThreads / 32) {
+    const int c = s_cnt[lane * Ep + x];
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
     }
-    s_tot[x] = run;
+    s_cnt[lane * Ep + x] = incl - c;
+    if (lane == 31) s_tot[x] = incl;
   }
   dev::cluster_sync();  // every CTA's totals are final and visible in the cluster
-  // 3. earlier CTAs' totals (the exclusive prefix) and all CTAs' (the arrivals)
+  // 3. earlier CTAs' totals (the exclusive prefix) and all CTAs' (the arrivals):
+  //    the cluster's (at most 16) remote loads issued before any is summed
   for (int x = tid; x < E; x += kAssignThreads) {
-    int before = 0, all = 0;
     const uint32_t addr = dev::smem_u32(s_tot + x);
-    for (int q = 0; q < nb; ++q) {
-      uint32_t remote;
-      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(q));
-      const int v = ld_cluster_s32(remote);
-      before += q < b ? v : 0;
-      all += v;
+    int v[kMaxAssignCtas];
+#pragma unroll
+    for (int q = 0; q < kMaxAssignCtas; ++q) {
+      v[q] = 0;
+      if (q < nb) {
+        uint32_t remote;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(q));
+        v[q] = ld_cluster_s32(remote);
+      }
+    }
+    int before = 0, all = 0;
+#pragma unroll
+    for (int q = 0; q < kMaxAssignCtas; ++q) {
+      before += q < b ? v[q] : 0;
+      all += v[q];
     }
     s_excl[x] = before;
     s_all[x] = all;
@@ -236,9 +252,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignA
     if (e < 0 || e >= E) e = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     int s = INT_MAX;
-    if (e >= 0) s = s_excl[e] + s_cnt[warp * E + e] + __popc(peers & lower);
+    if (e >= 0) s = s_excl[e] + s_cnt[warp * Ep + e] + __popc(peers & lower);
     __syncwarp();  // every peer has read the base before the leader moves it
-    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * E + e] += __popc(peers);
+    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * Ep + e] += __popc(peers);
     __syncwarp();
     if (in) {
       p.slot[a] = s;  // INT_MAX for an expert index outside [0, E)
@@ -336,7 +352,7 @@ int32_t launch_route_assign(const moe_config& c, const float* logits, const int3
 
 namespace {
 
-size_t assign_smem_bytes(int E) { return (32 + 3) * static_cast<size_t>(E) * sizeof(int); }
+size_t assign_smem_bytes(int E) { return (32 * static_cast<size_t>(E | 1) + 3 * E) * sizeof(int); }
 
 // CTAs in the assignment's cluster: 16 where the device co-schedules a
 // cluster of 16 such CTAs (a non-portable size), else the portable 8.

@@ -16,9 +16,9 @@
 //   whole waves (R = T / (2 * pairs * waves), rounded up to 8 rows): every SM
 //   streams the same share of x instead of a few SMs taking one tile more.
 // * Each CTA has two TMEM accumulators, so one tile's gate and top-k run
-//   while the next is loaded and multiplied, and eight epilogue warps, two
-//   per TMEM lane quarter: warp set h reads columns [h BN/2, (h+1) BN/2) of
-//   its 32 tokens, and set 1 hands its partial result to set 0 through
+//   while the next is loaded and multiplied, and sixteen epilogue warps, four
+//   per TMEM lane quarter: warp set h reads columns [h BN/4, (h+1) BN/4) of
+//   its 32 tokens, and sets 1-3 hand their partial results to set 0 through
 //   shared memory (a pair of mbarriers per accumulator, bounded waits).
 // * Each warp reads its logits from TMEM once (32-column chunks) and keeps a
 //   running maximum, the softmax denominator rescaled at each new maximum,
@@ -48,10 +48,10 @@ namespace {
 
 constexpr int kHalf = 128;                      // A rows of shared memory per CTA
 constexpr int kBK = 64, kUmmaK = 16;
-constexpr int kEpiWarps = 8;                    // two sets of four (one per TMEM lane quarter)
-constexpr int kThreads = 64 + 32 * kEpiWarps;   // 320
+constexpr int kSets = 4;                        // epilogue warp sets (column quarters)
+constexpr int kEpiWarps = 4 * kSets;            // one warp of each set per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // 576
 constexpr int kABytes = kHalf * kBK * 2;        // 16 KB
-constexpr int kNC = 32;                         // logits per TMEM load and chunk
 
 template <int BN>
 struct RCfg {
@@ -62,6 +62,7 @@ struct RCfg {
   static constexpr int kTmemCols = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
   static constexpr int kAccStride = kTmemCols / 2;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
+  static constexpr int kNC = BN / kSets >= 32 ? 32 : 16;  // logits per TMEM load and chunk
   static_assert(BN == 64 || BN == 128 || BN == 256, "N of the pair MMA");
   static_assert(kBBytes % 1024 == 0, "B stage alignment");
 };
@@ -87,16 +88,18 @@ struct TopState {
   int i2;
 };
 
-MOE_DEV float tree_max(float (&w)[kNC]) {
+template <int NC>
+MOE_DEV float tree_max(float (&w)[NC]) {
 #pragma unroll
-  for (int n = kNC / 2; n > 0; n >>= 1)
+  for (int n = NC / 2; n > 0; n >>= 1)
 #pragma unroll
     for (int i = 0; i < n; ++i) w[i] = fmaxf(w[i], w[i + n]);
   return w[0];
 }
-MOE_DEV int tree_min(int (&w)[kNC]) {
+template <int NC>
+MOE_DEV int tree_min(int (&w)[NC]) {
 #pragma unroll
-  for (int n = kNC / 2; n > 0; n >>= 1)
+  for (int n = NC / 2; n > 0; n >>= 1)
 #pragma unroll
     for (int i = 0; i < n; ++i) w[i] = min(w[i], w[i + n]);
   return w[0];
@@ -125,27 +128,27 @@ MOE_DEV void merge_above(TopState& a, float bm, float bs, int bi1, float bv2, in
   }
 }
 
-// Fold chunk v (columns e0 .. e0 + kNC - 1, all above the columns already
+// Fold chunk v (columns e0 .. e0 + NC - 1, all above the columns already
 // folded) into the running state.
-template <bool TWO>
-MOE_DEV void fold_chunk(TopState& st, const float (&v)[kNC], int e0) {
-  float w[kNC];
-  int id[kNC];
+template <bool TWO, int NC>
+MOE_DEV void fold_chunk(TopState& st, const float (&v)[NC], int e0) {
+  float w[NC];
+  int id[NC];
 #pragma unroll
-  for (int i = 0; i < kNC; ++i) w[i] = v[i];
-  const float cm = tree_max(w);
+  for (int i = 0; i < NC; ++i) w[i] = v[i];
+  const float cm = tree_max<NC>(w);
 #pragma unroll
-  for (int i = 0; i < kNC; ++i) id[i] = v[i] == cm ? i : kNC;
-  const int ci1 = tree_min(id);
+  for (int i = 0; i < NC; ++i) id[i] = v[i] == cm ? i : NC;
+  const int ci1 = tree_min<NC>(id);
   float cv2 = -INFINITY;
-  int ci2 = kNC;
+  int ci2 = NC;
   if (TWO) {
 #pragma unroll
-    for (int i = 0; i < kNC; ++i) w[i] = i == ci1 ? -INFINITY : v[i];
-    cv2 = tree_max(w);
+    for (int i = 0; i < NC; ++i) w[i] = i == ci1 ? -INFINITY : v[i];
+    cv2 = tree_max<NC>(w);
 #pragma unroll
-    for (int i = 0; i < kNC; ++i) id[i] = (i != ci1 && v[i] == cv2) ? i : kNC;
-    ci2 = tree_min(id);
+    for (int i = 0; i < NC; ++i) id[i] = (i != ci1 && v[i] == cv2) ? i : NC;
+    ci2 = tree_min<NC>(id);
   }
   float cs = 0.f;
   if (cm > -INFINITY) {
@@ -153,7 +156,7 @@ MOE_DEV void fold_chunk(TopState& st, const float (&v)[kNC], int e0) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < kNC; ++i) part[i & 7] += __expf(v[i] - cm);
+    for (int i = 0; i < NC; ++i) part[i & 7] += __expf(v[i] - cm);
     cs = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
   }
   merge_above<TWO>(st, cm, cs, e0 + ci1, cv2, e0 + ci2);
@@ -173,7 +176,7 @@ router_topk_pair_kernel(const __grid_constant__ CUtensorMap tmX,
   __shared__ volatile int s_abort;
   __shared__ float s_bias[BN];
   __shared__ uint64_t part_full[2], part_empty[2];  // set 1 -> set 0 handoff, per accumulator
-  __shared__ TopState s_part[2][kHalf];
+  __shared__ TopState s_part[2][kSets - 1][kHalf];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -196,8 +199,8 @@ router_topk_pair_kernel(const __grid_constant__ CUtensorMap tmX,
     for (int a = 0; a < 2; ++a) {
       dev::mbar_init(&tfull_bar[a], 1);
       dev::mbar_init(&tempty_bar[a], 2 * kEpiWarps);  // one arrival per epilogue warp, both CTAs
-      dev::mbar_init(&part_full[a], 4 * 32);           // set 1's threads
-      dev::mbar_init(&part_empty[a], 4 * 32);          // set 0's threads
+      dev::mbar_init(&part_full[a], (kSets - 1) * 4 * 32);  // sets 1..3's threads
+      dev::mbar_init(&part_empty[a], 4 * 32);               // set 0's threads
     }
     dev::mbar_init(&done_bar, 1);
     dev::fence_mbar_init();
@@ -287,14 +290,15 @@ router_topk_pair_kernel(const __grid_constant__ CUtensorMap tmX,
   } else {
     // ---------------- epilogue: warps 2..9 ----------------
     const int q = warp & 3;          // TMEM lane quarter this warp may read
-    const int h = (warp - 2) >> 2;   // column half: [h BN/2, (h+1) BN/2)
+    const int h = (warp - 2) >> 2;   // column quarter: [h BN/4, (h+1) BN/4)
     const int row_local = q * 32 + lane;
     // the bias, off the producer's path (named barrier 1: the 256 epilogue threads)
     for (int i = tid - 64; i < BN; i += kThreads - 64)
       s_bias[i] = (p.bias && i < p.E) ? p.bias[i] : 0.f;
     asm volatile("bar.sync 1, %0;" ::"n"(kThreads - 64) : "memory");
-    const int c_lo = h * (BN / 2);
-    const int c_hi = min(c_lo + BN / 2, p.E);
+    constexpr int NC = C::kNC;
+    const int c_lo = h * (BN / kSets);
+    const int c_hi = min(c_lo + BN / kSets, p.E);
     const uint32_t tempty0 = dev::mapa(&tempty_bar[0], 0), tempty1 = dev::mapa(&tempty_bar[1], 0);
     const bool two = p.topk == 2;
     int acc = 0;
@@ -309,43 +313,49 @@ router_topk_pair_kernel(const __grid_constant__ CUtensorMap tmX,
                              static_cast<uint32_t>(acc * C::kAccStride);
       TopState st{-INFINITY, 0.f, INT_MAX, -INFINITY, INT_MAX};
 #pragma unroll 1
-      for (int e0 = c_lo; e0 < c_hi; e0 += kNC) {
-        uint32_t r[kNC];
-        dev::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(e0), r);
+      for (int e0 = c_lo; e0 < c_hi; e0 += NC) {
+        uint32_t r[NC];
+        if constexpr (NC == 32) dev::tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(e0), r);
+        else dev::tmem_ld_32x32b_x16(tbase + static_cast<uint32_t>(e0), r);
         dev::tmem_wait_ld();
-        float v[kNC];
-        if (e0 + kNC <= c_hi) {
+        float v[NC];
+        if (e0 + NC <= c_hi) {
 #pragma unroll
-          for (int i = 0; i < kNC; ++i) v[i] = __uint_as_float(r[i]) + s_bias[e0 + i];
+          for (int i = 0; i < NC; ++i) v[i] = __uint_as_float(r[i]) + s_bias[e0 + i];
         } else {  // the last, partial chunk: columns past E take no part
 #pragma unroll
-          for (int i = 0; i < kNC; ++i)
+          for (int i = 0; i < NC; ++i)
             v[i] = e0 + i < c_hi ? __uint_as_float(r[i]) + s_bias[e0 + i] : -INFINITY;
         }
-        if (two) fold_chunk<true>(st, v, e0);
-        else fold_chunk<false>(st, v, e0);
+        if (two) fold_chunk<true, NC>(st, v, e0);
+        else fold_chunk<false, NC>(st, v, e0);
       }
       // the accumulator is free for the tile after next
       dev::tc_fence_before();
       __syncwarp();
       if (lane == 0) dev::mbar_arrive_cluster(acc ? tempty1 : tempty0);
-      // set 1 -> set 0: slot `acc` of the handoff, its (acc_phase)-th use
-      if (h == 1) {
+      // sets 1..3 -> set 0: slot `acc` of the handoff, its (acc_phase)-th use
+      if (h > 0) {
         ok = 0;
         if (lane == 0) ok = dev::mbar_wait(&part_empty[acc], acc_phase ^ 1u, ab) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        s_part[acc][row_local] = st;
+        s_part[acc][h - 1][row_local] = st;
         dev::mbar_arrive(&part_full[acc]);
       } else {
         ok = 0;
         if (lane == 0) ok = dev::mbar_wait(&part_full[acc], acc_phase, ab) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        const TopState o = s_part[acc][row_local];
+        TopState o[kSets - 1];
+#pragma unroll
+        for (int j = 0; j < kSets - 1; ++j) o[j] = s_part[acc][j][row_local];
         dev::mbar_arrive(&part_empty[acc]);
-        if (two) merge_above<true>(st, o.m, o.s, o.i1, o.v2, o.i2);
-        else merge_above<false>(st, o.m, o.s, o.i1, o.v2, o.i2);
+#pragma unroll
+        for (int j = 0; j < kSets - 1; ++j) {  // quarters in increasing column order
+          if (two) merge_above<true>(st, o[j].m, o[j].s, o[j].i1, o[j].v2, o[j].i2);
+          else merge_above<false>(st, o[j].m, o[j].s, o[j].i1, o[j].v2, o[j].i2);
+        }
         const int tok = t * 2 * R + static_cast<int>(rank) * R + row_local;
         if (row_local < R && tok < p.T) {
           const float inv = 1.0f / st.s;  // gate of the maximum: exp(m - m) / sum
