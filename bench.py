@@ -40,7 +40,7 @@ FFN_TRAFFIC = {
     "switch_base": (1240.836e6 + 29.177e6, "profiles/ffn_tc_switch_base.md"),
     "xmoe_top2": (604.122e6 + 228.916e6 + 825.805e6 + 55.799e6, "profiles/gemm_pair_xmoe_top2.md"),
     # captured on 8 experts (same capacity and per-expert load), scaled by 64 / 8
-    "pangu_rre": ((1180.756e6 + 101.806e6) * 8, "profiles/ffn_pair_pangu_rre.md"),
+    "pangu_rre": ((1194.575e6 + 103.069e6) * 8, "profiles/ffn_pair_pangu_rre.md"),
 }
 METRIC = "MoE-layer tokens/sec (1 B200); expert-FFN TFLOP/s; dispatch+combine GB/s"
 

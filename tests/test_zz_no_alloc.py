@@ -6,7 +6,8 @@ The entry point keeps its partial sums in a fixed array inside the library
 instead of a caller workspace.  This test calls it through the C ABI twice in
 a row, on different gradients, and checks each result against the
 workspace-taking sparseclip_norm on the same inputs and against the CPU
-oracle's norm.  It lives in its own file
+oracle's norm; the device's free memory is the same before and after the
+second call.  It lives in its own file
 that pytest collects last and passes alone in a fresh process as well as
 after the other tests.
 """
@@ -54,11 +55,15 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
         (_grads(1, dev, 300, [1_000_003, 5, 4096]), 64),  # several launches, ragged tails
         (_grads(2, dev, 64, [777_777]), 8),               # second call, other data and E
     ]
-    for (dense, sparse), E in cases:
+    for i, ((dense, sparse), E) in enumerate(cases):
         ref = moe.sparseclip_norm(dense, sparse, E)
         out = torch.full((3,), float("nan"), dtype=torch.float64, device=dev)
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info(dev)[0]
         assert _noalloc(moe, dense, sparse, E, out) == 0, moe.lib.moe_last_error()
         torch.cuda.synchronize()
+        if i > 0:  # (the first call may load the kernels' module)
+            assert torch.cuda.mem_get_info(dev)[0] == free_before, "the call allocated device memory"
         got, want = out.cpu(), ref.cpu()
         assert bool(((got - want).abs() <= RTOL * want.abs()).all()), (got, want)
         norm = oracle.sparseclip_norm([t.cpu() for t in dense], [t.cpu() for t in sparse], E)
