@@ -10,7 +10,9 @@
 // Pass 1 (HBM-bound: reads the logits once): a warp per token, the logits of
 // four tokens per warp loaded before any is reduced, E <= 256 logits held 8
 // per lane (coalesced); max/argmax and the softmax sum by shuffles; each lane
-// accumulates p for its experts in double across the warp's tokens, the
+// accumulates p for its experts in fp32 over groups of 16 tokens and adds each
+// group's sums to its double sums in shared memory (one conversion per 16
+// tokens), the
 // argmax is counted in shared memory, H(p) = ln(s) - sum_e p_e (h_e - m) per
 // token.  Each block (three per SM, one wave) writes its partial P[E], counts[E]
 // and entropy sum.  Pass 2: a block per expert adds that expert's partials
@@ -29,6 +31,7 @@ constexpr int kAuxThreads = 256;  // 8 warps
 constexpr int kAuxWarps = kAuxThreads / 32;
 constexpr int kAuxInFlight = 4;  // tokens per warp whose logits are loaded together
 constexpr int kAuxBlocksPerSm = 3;  // 3 x 256 threads x <= 85 registers fill the register file
+constexpr int kAuxGroup = 16;       // tokens summed in fp32 before each double add
 
 __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kernel(
     int64_t T, int E, const float* __restrict__ logits, double* __restrict__ part_P,
@@ -40,9 +43,12 @@ __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kern
   dev::pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < 256; e += kAuxThreads) s_cnt[e] = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) s_P[warp][lane + 32 * q] = 0.0;  // this lane's double sums
   if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // pass 2's finishing counter
   __syncthreads();
-  double accP[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float grpP[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int in_grp = 0;
   double accH = 0.0;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kAuxWarps;
   // one token's logits, lane + 32 q for q < 8 (-inf past E)
@@ -77,7 +83,7 @@ __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kern
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const bool in = lane + 32 * q < E;
-      ex[q] = in ? expf(v[q] - m) : 0.f;
+      ex[q] = in ? __expf(v[q] - m) : 0.f;
       s += ex[q];
       w += in ? ex[q] * (v[q] - m) : 0.f;
     }
@@ -88,7 +94,15 @@ __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kern
     }
     const float inv = 1.0f / s;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) accP[q] += static_cast<double>(ex[q] * inv);
+    for (int q = 0; q < 8; ++q) grpP[q] += ex[q] * inv;
+    if (++in_grp == kAuxGroup) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        s_P[warp][lane + 32 * q] += static_cast<double>(grpP[q]);
+        grpP[q] = 0.f;
+      }
+      in_grp = 0;
+    }
     if (lane == 0) {
       if (bi < E) atomicAdd(&s_cnt[bi], 1);
       // H = -sum p ln p = ln s - sum p (h - m)
@@ -110,7 +124,7 @@ __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kern
     token(v);
   }
 #pragma unroll
-  for (int q = 0; q < 8; ++q) s_P[warp][lane + 32 * q] = accP[q];
+  for (int q = 0; q < 8; ++q) s_P[warp][lane + 32 * q] += static_cast<double>(grpP[q]);
   if (lane == 0) s_H[warp] = accH;
   __syncthreads();
   double* outP = part_P + static_cast<int64_t>(blockIdx.x) * E;

@@ -36,6 +36,7 @@ namespace {
 
 constexpr int kAssignThreads = 1024;
 constexpr int kMaxAssignCtas = 16;  // CTAs in the assignment's cluster (16 or 8)
+constexpr int kMaxRounds = 8;       // rounds of 32 choices per warp held in registers
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t t) {
   // output #t of splitmix64 seeded with `seed` (Steele, Lea & Flood 2014)
@@ -193,15 +194,41 @@ __global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignA
   dev::pdl_wait();  // the choices come from the previous kernel
   __syncthreads();
 
-  // 1. this warp's counts per expert (the leader of each group of peers adds)
+  // 1. this warp's counts per expert (the leader of each group of peers adds).
+  //    Runs of up to kMaxRounds rounds keep each lane's choices and their
+  //    offsets within the warp's run in registers for step 4.
+  const bool in_regs = p.per_warp <= 32 * kMaxRounds;  // the same for every warp
+  int ev[kMaxRounds], lv[kMaxRounds];
+  if (in_regs) {
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {  // all loads first
+      const int64_t a = w0 + 32 * r + lane;
+      ev[r] = a < w1 ? __ldg(p.expert_idx + a) : -1;
+      if (ev[r] < 0 || ev[r] >= E) ev[r] = -1;
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+      lv[r] = 0;
+      if (w0 + 32 * r < w1) {  // the same for the whole warp
+        const int e = ev[r];
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int base = e >= 0 ? s_cnt[warp * Ep + e] : 0;
+        __syncwarp();  // every peer has read the base before the leader moves it
+        if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * Ep + e] = base + __popc(peers);
+        __syncwarp();
+        lv[r] = base + __popc(peers & lower);
+      }
+    }
+  } else {
 #pragma unroll 4
-  for (int64_t base = w0; base < w1; base += 32) {
-    const int64_t a = base + lane;
-    int e = a < w1 ? __ldg(p.expert_idx + a) : -1;
-    if (e < 0 || e >= E) e = -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * Ep + e] += __popc(peers);
-    __syncwarp();  // the next round's leader may be another lane
+    for (int64_t base = w0; base < w1; base += 32) {
+      const int64_t a = base + lane;
+      int e = a < w1 ? __ldg(p.expert_idx + a) : -1;
+      if (e < 0 || e >= E) e = -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) s_cnt[warp * Ep + e] += __popc(peers);
+      __syncwarp();  // the next round's leader may be another lane
+    }
   }
   __syncthreads();
   // 2. exclusive prefix over the warps (choice order), CTA totals: a warp per
@@ -244,8 +271,22 @@ __global__ void __launch_bounds__(kAssignThreads, 1) assign_kernel(const AssignA
   dev::cluster_sync();  // no CTA reads another's shared memory after this (it may exit)
 
   // 4. slots in choice order
+  if (in_regs) {
+#pragma unroll
+    for (int r = 0; r < kMaxRounds; ++r) {
+      const int64_t a = w0 + 32 * r + lane;
+      if (a < w1) {
+        const int e = ev[r];
+        const int s = e >= 0 ? s_excl[e] + s_cnt[warp * Ep + e] + lv[r] : INT_MAX;
+        p.slot[a] = s;  // INT_MAX for an expert index outside [0, E)
+        const bool kp = e >= 0 && s < p.C;
+        p.kept[a] = kp ? 1 : 0;
+        if (kp) p.tok_of_row[static_cast<int64_t>(e) * p.C + s] = static_cast<int32_t>(a / p.k);
+      }
+    }
+  }
 #pragma unroll 4
-  for (int64_t base = w0; base < w1; base += 32) {
+  for (int64_t base = in_regs ? w1 : w0; base < w1; base += 32) {
     const int64_t a = base + lane;
     const bool in = a < w1;
     int e = in ? __ldg(p.expert_idx + a) : -1;

@@ -441,6 +441,8 @@ SMALL = [
     ("tiny_fp32_top2", 400, 32, 48, 8, 2, 1.5, "topk", 1, 0.0),
     ("odd_experts_top2", 500, 64, 128, 40, 2, 1.0, "topk", 1, 0.0),
     ("seven_experts", 300, 128, 64, 7, 1, 1.0, "topk", 1, 0.0),
+    # 140000 choices: more than the slot assignment keeps in registers (two passes)
+    ("many_choices_top2", 70000, 64, 64, 16, 2, 1.0, "topk", 1, 0.0),
     # GEGLU experts in each FFN kernel: fused (C = 62), two launches (C = 300), SM pairs (C = 550)
     ("geglu_top1", 1000, 128, 256, 16, 1, 1.0, "topk", 1, 0.0),
     ("geglu_top2_multi_block", 1200, 128, 128, 8, 2, 2.0, "topk", 1, 0.0),
