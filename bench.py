@@ -251,7 +251,8 @@ def kernel_launches(w, C):
     else:
         route = 3                       # fp32 router, gate/top-k, slot assignment
     # bf16: one persistent kernel for both GEMMs when C <= 128 (single CTAs) or
-    # C >= 512 (SM pairs); two grouped launches in between; fp32: two FMA GEMMs
+    # C >= 512 with d_model >= 2048 (SM pairs); two grouped launches otherwise;
+    # fp32: two FMA GEMMs
     ffn = 1 if (bf16 and (C <= 128 or (C >= 512 and w.d_model >= 2048))) else 2
     combine = 0 if (bf16 and w.k == 1) else 1   # top-1 bf16: inside the FFN's GEMM 2
     return route + 1 + ffn + combine
