@@ -20,17 +20,17 @@
 //   per TMEM lane quarter: warp set h reads columns [h BN/4, (h+1) BN/4) of
 //   its 32 tokens, and sets 1-3 hand their partial results to set 0 through
 //   shared memory (a pair of mbarriers per accumulator, bounded waits).
-// * Each warp reads its logits from TMEM once (32-column chunks) and keeps a
-//   running maximum, the softmax denominator rescaled at each new maximum,
-//   and the running top-1 / top-2 with their indices; inside a chunk the
-//   maximum, second and their lowest columns come from pairwise trees.
-//   Chunks and the two halves are combined in increasing e, and a later part
-//   replaces a kept entry only when strictly larger, which gives the (value
-//   desc, index asc) order of the top-k definition.
+// * Each warp reads its logits from TMEM once (chunks of 32 columns, 16 when
+//   E <= 64) and keeps a running maximum, the softmax denominator rescaled at
+//   each new maximum, and the running top-1 / top-2 with their indices;
+//   inside a chunk the maximum, second and their lowest columns come from
+//   pairwise trees.  Chunks and the four quarters are combined in increasing
+//   e, and a later part replaces a kept entry only when strictly larger, which
+//   gives the (value desc, index asc) order of the top-k definition.
 //
 // Roles: warp 0 lane 0 of each CTA loads its halves with TMA (both CTAs'
 // copies complete on CTA 0's "full" barrier); warp 1 lane 0 of CTA 0 issues
-// the MMAs and commits them to both CTAs' barriers; warps 2-9 drain TMEM.
+// the MMAs and commits them to both CTAs' barriers; warps 2-17 drain TMEM.
 // Every wait is bounded and shares the call's give-up signal; a cluster
 // barrier brackets the kernel so neither CTA frees TMEM or exits while its
 // partner may still use it.  TMA loads fill only the issuing CTA's own
@@ -288,7 +288,7 @@ router_topk_pair_kernel(const __grid_constant__ CUtensorMap tmX,
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..9 ----------------
+    // ---------------- epilogue: warps 2..17 ----------------
     const int q = warp & 3;          // TMEM lane quarter this warp may read
     const int h = (warp - 2) >> 2;   // column quarter: [h BN/4, (h+1) BN/4)
     const int row_local = q * 32 + lane;
