@@ -7,14 +7,13 @@
 // with p(x) the softmax of eq. (1) over all E experts and the argmax taken on
 // the fp32 logits, ties to the lower index (the top-1 choice).
 //
-// Pass 1 (HBM-bound: reads the logits once): a warp per token, the logits of
-// four tokens per warp loaded before any is reduced, E <= 256 logits held 8
-// per lane (coalesced); max/argmax and the softmax sum by shuffles; each lane
+// Pass 1 (reads the logits once): a warp per token, the logits of two tokens
+// per warp loaded before either is reduced, E <= 256 logits held 8 per lane
+// (coalesced); max/argmax and the softmax sum by shuffles; each lane
 // accumulates p for its experts in fp32 over groups of 16 tokens and adds each
 // group's sums to its double sums in shared memory (one conversion per 16
-// tokens), the
-// argmax is counted in shared memory, H(p) = ln(s) - sum_e p_e (h_e - m) per
-// token.  Each block (three per SM, one wave) writes its partial P[E], counts[E]
+// tokens), the argmax is counted in shared memory, and H(p) = ln(s) -
+// sum_e p_e (h_e - m) per token.  Each block (four per SM, one wave) writes its partial P[E], counts[E]
 // and entropy sum.  Pass 2: a block per expert adds that expert's partials
 // (strided, then a fixed tree: deterministic); the last block to finish
 // (a counter that pass 1 zeroes) forms sum_e f_e P_e and the entropy, in a
@@ -29,8 +28,8 @@ namespace {
 
 constexpr int kAuxThreads = 256;  // 8 warps
 constexpr int kAuxWarps = kAuxThreads / 32;
-constexpr int kAuxInFlight = 4;  // tokens per warp whose logits are loaded together
-constexpr int kAuxBlocksPerSm = 3;  // 3 x 256 threads x <= 85 registers fill the register file
+constexpr int kAuxInFlight = 2;  // tokens per warp whose logits are loaded together
+constexpr int kAuxBlocksPerSm = 4;  // 4 x 256 threads x <= 64 registers fill the register file
 constexpr int kAuxGroup = 16;       // tokens summed in fp32 before each double add
 
 __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kernel(
