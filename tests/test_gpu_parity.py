@@ -443,6 +443,12 @@ SMALL = [
     ("seven_experts", 300, 128, 64, 7, 1, 1.0, "topk", 1, 0.0),
     # 140000 choices: more than the slot assignment keeps in registers (two passes)
     ("many_choices_top2", 70000, 64, 64, 16, 2, 1.0, "topk", 1, 0.0),
+    # E = 200 of the router's 256 columns: the last chunk is partial and falls in
+    # the fourth column quarter (5000 tokens: the first top-3 logit gap below
+    # 1e-5, where fp32 and fp64 routing may part, is at token 5805)
+    ("e200_top2", 5000, 128, 64, 200, 2, 1.0, "topk", 1, 0.0),
+    # every token's first choice is expert 0 (one expert takes T choices)
+    ("hot_e256_top2", 20000, 64, 64, 256, 2, 2.0, "topk", 1, 100.0),
     # GEGLU experts in each FFN kernel: fused (C = 62), two launches (C = 300), SM pairs (C = 550)
     ("geglu_top1", 1000, 128, 256, 16, 1, 1.0, "topk", 1, 0.0),
     ("geglu_top2_multi_block", 1200, 128, 128, 8, 2, 2.0, "topk", 1, 0.0),
