@@ -25,7 +25,6 @@
 #include <cuda.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -400,41 +399,6 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
   }
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-int32_t make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
-  return MOE_OK;
-}
-
 }  // namespace
 
 // tile counter, then one counter per (expert, chunk of at most 256 rows)
@@ -475,10 +439,10 @@ int32_t launch_ffn_tc(const moe_config& c, const void* xe, const void* W1, const
   const bool glu = c.expert == MOE_EXPERT_GEGLU;
   const int64_t n1 = glu ? 2 * f : f;  // W1 rows per expert
   CUtensorMap tx, tw1, th, tw2;
-  int32_t rc = make_tmap(&tx, xe, static_cast<uint64_t>(E * C), static_cast<uint64_t>(d), kBM);
-  if (rc == MOE_OK) rc = make_tmap(&tw1, W1, static_cast<uint64_t>(E * n1), static_cast<uint64_t>(d), kBN);
-  if (rc == MOE_OK) rc = make_tmap(&th, H, static_cast<uint64_t>(E * C), static_cast<uint64_t>(f), kBM);
-  if (rc == MOE_OK) rc = make_tmap(&tw2, W2, static_cast<uint64_t>(E * d), static_cast<uint64_t>(f), kBN);
+  int32_t rc = make_tmap_bf16(&tx, xe, static_cast<uint64_t>(E * C), static_cast<uint64_t>(d), kBM);
+  if (rc == MOE_OK) rc = make_tmap_bf16(&tw1, W1, static_cast<uint64_t>(E * n1), static_cast<uint64_t>(d), kBN);
+  if (rc == MOE_OK) rc = make_tmap_bf16(&th, H, static_cast<uint64_t>(E * C), static_cast<uint64_t>(f), kBM);
+  if (rc == MOE_OK) rc = make_tmap_bf16(&tw2, W2, static_cast<uint64_t>(E * d), static_cast<uint64_t>(f), kBN);
   if (rc != MOE_OK) return rc;
   const int64_t mblk_max = (C + kBM - 1) / kBM;
   const int64_t nb1 = (n1 + kBN - 1) / kBN, nb2 = (d + kBN - 1) / kBN;

@@ -22,7 +22,6 @@
 #include <cuda.h>
 
 #include <climits>
-#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -329,51 +328,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 // ---- host side ----------------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor [rows, cols] (row-major), box [box_rows, 64], 128-byte swizzle.
-int32_t make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
-  return MOE_OK;
-}
-
 template <int BN, int EPI>
 int32_t launch_gemm(const void* A, uint64_t a_rows, const void* B, uint64_t b_rows,
                     const GemmParams& p, int64_t max_tiles, cudaStream_t s) {
   using C = Cfg<BN>;
   if (max_tiles <= 0) return MOE_OK;
   CUtensorMap ta, tb;
-  int32_t rc = make_tmap(&ta, A, a_rows, static_cast<uint64_t>(p.K), kBM);
+  int32_t rc = make_tmap_bf16(&ta, A, a_rows, static_cast<uint64_t>(p.K), kBM);
   if (rc != MOE_OK) return rc;
-  rc = make_tmap(&tb, B, b_rows, static_cast<uint64_t>(p.K), BN);
+  rc = make_tmap_bf16(&tb, B, b_rows, static_cast<uint64_t>(p.K), BN);
   if (rc != MOE_OK) return rc;
   auto kern = gemm_tc_kernel<BN, EPI>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=

@@ -64,6 +64,9 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // ---- internal launchers (defined in the .cu files) ---------------------------
 
+// 2-D bf16 [rows, cols] tensor map, boxes of box_rows x 64 (128-byte swizzle)
+int32_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows);
 int32_t launch_router_tc(const moe_config& c, const void* x, const void* Wr, const float* bias,
                          float* logits, int32_t* status, cudaStream_t s);
 int32_t launch_router_f32(const moe_config& c, const void* x, const void* Wr, const float* bias,

@@ -384,42 +384,6 @@ router_topk_pair_kernel(const __grid_constant__ CUtensorMap tmX,
   }
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// bf16 [rows, cols] row-major, box [box_rows, 64], 128-byte swizzle; rows past
-// the end read as zero
-int32_t make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
-  return MOE_OK;
-}
 
 // Resident pairs of one kernel on this device, queried once per (device, kernel).
 template <int BN>
@@ -474,10 +438,10 @@ int32_t launch_router_pair(const moe_config& c, const void* x, const void* Wr, R
   p.R = static_cast<int32_t>(R);
   p.tiles = static_cast<int32_t>((T + 2 * R - 1) / (2 * R));
   CUtensorMap tx, tw;
-  rc = make_tmap(&tx, x, static_cast<uint64_t>(c.T), static_cast<uint64_t>(c.d_model),
+  rc = make_tmap_bf16(&tx, x, static_cast<uint64_t>(c.T), static_cast<uint64_t>(c.d_model),
                  static_cast<uint32_t>(R));
   if (rc != MOE_OK) return rc;
-  rc = make_tmap(&tw, Wr, static_cast<uint64_t>(c.E), static_cast<uint64_t>(c.d_model),
+  rc = make_tmap_bf16(&tw, Wr, static_cast<uint64_t>(c.E), static_cast<uint64_t>(c.d_model),
                  static_cast<uint32_t>(C::kBRows));
   if (rc != MOE_OK) return rc;
   auto kern = router_topk_pair_kernel<BN>;
