@@ -19,9 +19,10 @@
 //      giving the CTA's per-expert total; cluster barrier;
 //   3. each CTA reads every CTA's totals (DSMEM): the sum over earlier CTAs
 //      is its exclusive prefix, the sum over all the arrivals; barrier;
-//   4. each warp walks its run again: slot = earlier CTAs + earlier warps +
-//      earlier rounds of this warp + rank among this round's peers;
-//      kept = slot < C, and the row -> token map;
+//   4. slot = earlier CTAs + earlier warps + earlier rounds of this warp +
+//      rank among this round's peers (the last two kept in registers from
+//      step 1 when a warp's run is at most 8 rounds, else found by walking
+//      the run again); kept = slot < C, and the row -> token map;
 //   5. CTA 0 writes arrivals, kept counts and the dropped total; every CTA
 //      marks the free rows of its share of experts with -1.
 #include <algorithm>
