@@ -58,7 +58,7 @@ typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 enum moe_error {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARGUMENT = -1, /* null pointer, bad size, bad enum value   */
-  MOE_ERR_UNSUPPORTED = -2,      /* valid MoE, but outside this build's range */
+  MOE_ERR_UNSUPPORTED = -2,      /* valid MoE, but outside this library's range */
   MOE_ERR_ALIGNMENT = -3,        /* pointer not 16-byte aligned               */
   MOE_ERR_WORKSPACE = -4,        /* workspace missing or too small            */
   MOE_ERR_CUDA = -5              /* a CUDA runtime / driver call failed       */
@@ -155,10 +155,10 @@ uint64_t moe_wait_limit_ns(void);
  * Returns -1 if E < 1, T < 0 or capacity_factor < 0. */
 int32_t moe_capacity(int64_t T, int32_t E, double capacity_factor);
 
-/* MOE_OK if `cfg` is a layer this build runs, else the error code. */
+/* MOE_OK if `cfg` is a layer this library runs, else the error code. */
 int32_t moe_config_check(const moe_config* cfg);
 
-/* Bytes of scratch moe_topk_assign needs (0 if cfg is invalid).  This build's
+/* Bytes of scratch moe_topk_assign needs (0 if cfg is invalid).  The library's
  * assignment exchanges its counts on chip and needs none: 0 for every cfg. */
 size_t moe_assign_workspace_size(const moe_config* cfg);
 
