@@ -210,6 +210,9 @@ FFN_SHAPES = {
     "sm_pairs_fused": (4, 600, 2048, 256, [600, 1, 513, 256]),
     # the same kernel: token chunks of every size class, GEMM-1 feature blocks cut short
     "sm_pairs_fused_chunks": (6, 560, 2048, 320, [1, 17, 255, 257, 513, 560]),
+    # the same kernel: rest chunks of 18 .. 64 rows after one or two full chunks
+    # (N = 32 or 64; 274 rows: a rest of 18 in a 32-column tile)
+    "sm_pairs_fused_rest": (6, 576, 2048, 256, [288, 320, 544, 576, 530, 274]),
     # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
     "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
 }
@@ -453,6 +456,9 @@ SMALL = [
     ("geglu_top1", 1000, 128, 256, 16, 1, 1.0, "topk", 1, 0.0),
     ("geglu_top2_multi_block", 1200, 128, 128, 8, 2, 2.0, "topk", 1, 0.0),
     ("geglu_rre_pairs", 4400, 64, 128, 8, 1, 1.0, "rre", 2, 0.0),
+    # top-1 on the fused SM-pair FFN (d >= 2048, C = 550): GEMM 2 writes gate * row
+    # to y in token order, experts over 512 rows with a rest chunk
+    ("pairs_fused_top1", 4400, 2048, 256, 8, 1, 1.0, "topk", 1, 0.0),
 ]
 
 
