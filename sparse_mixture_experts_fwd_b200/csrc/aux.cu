@@ -14,7 +14,7 @@
 // group's sums to its double sums in shared memory (one conversion per 16
 // tokens), the argmax is counted in shared memory, and H(p) = ln(s) -
 // sum_e p_e (h_e - m) per token.  Each block (four per SM, one wave) writes its partial P[E], counts[E]
-// and entropy sum.  Pass 2: a block per expert adds that expert's partials
+// and entropy sum, expert-major.  Pass 2: a block per expert adds that expert's partials
 // (strided, then a fixed tree: deterministic); the last block to finish
 // (a counter that pass 1 zeroes) forms sum_e f_e P_e and the entropy, in a
 // fixed order.
@@ -126,13 +126,12 @@ __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kern
   for (int q = 0; q < 8; ++q) s_P[warp][lane + 32 * q] += static_cast<double>(grpP[q]);
   if (lane == 0) s_H[warp] = accH;
   __syncthreads();
-  double* outP = part_P + static_cast<int64_t>(blockIdx.x) * E;
-  int32_t* outC = part_cnt + static_cast<int64_t>(blockIdx.x) * E;
+  // expert-major partials: pass 2's block for expert e reads its row coalesced
   for (int e = threadIdx.x; e < E; e += kAuxThreads) {
     double sum = 0.0;
     for (int wq = 0; wq < kAuxWarps; ++wq) sum += s_P[wq][e];
-    outP[e] = sum;
-    outC[e] = s_cnt[e];
+    part_P[static_cast<int64_t>(e) * gridDim.x + blockIdx.x] = sum;
+    part_cnt[static_cast<int64_t>(e) * gridDim.x + blockIdx.x] = s_cnt[e];
   }
   if (threadIdx.x == 0) {
     double sum = 0.0;
@@ -141,7 +140,8 @@ __global__ void __launch_bounds__(kAuxThreads, kAuxBlocksPerSm) aux_partial_kern
   }
 }
 
-// Pass 2: block e adds expert e's partials over the pass-1 blocks (thread i
+// Pass 2: block e adds expert e's partials over the pass-1 blocks, stored
+// expert-major (thread i
 // takes blocks i, i + 256, ..., then a fixed tree), f_e = count / T,
 // P_e = sum / T, fe_Pe[e] = f_e * P_e.  The block that finishes last (by the
 // counter pass 1 zeroed) forms loss = alpha * E * sum_e f_e P_e and
@@ -163,9 +163,11 @@ __global__ void __launch_bounds__(256, 1) aux_reduce_kernel(int64_t T, int E, in
   const int e = blockIdx.x;
   double p = 0.0;
   long long c = 0;
+  const double* rowP = part_P + static_cast<int64_t>(e) * nblk;
+  const int32_t* rowC = part_cnt + static_cast<int64_t>(e) * nblk;
   for (int b = threadIdx.x; b < nblk; b += 256) {
-    p += part_P[static_cast<int64_t>(b) * E + e];
-    c += part_cnt[static_cast<int64_t>(b) * E + e];
+    p += rowP[b];
+    c += rowC[b];
   }
   s_p[threadIdx.x] = p;
   s_c[threadIdx.x] = c;
@@ -217,7 +219,7 @@ int aux_blocks(const moe_config& c) {
 
 }  // namespace
 
-// per block: P [E] double, counts [E] int32; then the entropy sums [nblk]
+// per expert: P [nblk] double, then counts [nblk] int32 (expert-major); then the entropy sums [nblk]
 // double; then f_e P_e [E] double; then pass 2's finishing counter
 size_t aux_workspace_bytes(const moe_config& c) {
   const size_t nblk = static_cast<size_t>(aux_blocks(c));
