@@ -215,7 +215,31 @@ FFN_SHAPES = {
     "sm_pairs_fused_rest": (6, 576, 2048, 256, [288, 320, 544, 576, 530, 274]),
     # C <= 128: the fused persistent kernel (both GEMMs, per-expert dependency counters)
     "single_block": (40, 100, 256, 512, [100, 0, 1, 37, 64, 99] * 6 + [100, 100, 0, 5]),
+    # E = 256, the most experts each kernel's scheduling tables hold: the two-launch
+    # SM-pair GEMMs (d < 2048) and the one-launch SM-pair kernel (d = 2048, 512 units)
+    "sm_pairs_e256": (256, 512, 256, 64, [0, 1, 17, 255, 256, 257, 300, 511, 512] * 28 + [512] * 4),
+    "sm_pairs_fused_e256": (256, 512, 2048, 64, [0, 1, 17, 255, 256, 257, 300, 511, 512] * 28 + [512] * 4),
 }
+
+
+class FarCount:
+    """Elements beyond 2^-7 relative + 1e-3 absolute of the oracle, pooled over
+    every checked row of a call: the rate is a property of the arithmetic, and
+    an expert of a few rows holds too few elements to estimate it alone (at a
+    0.11 % rate, 3 or more beyond among the 1088 elements of a 17-row H with
+    f = 64 has a probability of about 0.12; with 256 experts some expert sees it)."""
+
+    def __init__(self):
+        self.n = 0
+        self.total = 0
+
+    def add(self, a, b):
+        self.n += int(((a.double() - b.double()).abs() > 2.0 ** -7 * b.double().abs() + 1e-3).sum())
+        self.total += a.numel()
+
+    def check(self, rate):
+        if self.total:
+            assert self.n / self.total < rate, f"{self.n} of {self.total} elements beyond 2^-7 rel + 1e-3"
 
 
 @pytest.mark.parametrize("shape", sorted(FFN_SHAPES))
@@ -238,21 +262,21 @@ def test_expert_ffn_ragged_tiles(moe, cuda_device, dtype, shape):
     assert int(st.item()) == 0
     ye_ref, H_ref = oracle.expert_ffn(xe, W1, W2, kept, with_H=True, nthreads=threads())
     H, ye = H.cpu(), ye.cpu()
+    far = FarCount()
     for e in range(E):
         n = int(kept[e])
         if dtype == torch.bfloat16:
             assert_close(H[e, :n], H_ref[e, :n], what=f"H[{e}]")
             assert_close(ye[e, :n], ye_ref[e, :n], what=f"ye[{e}]")
-            # beyond the stated tolerance: rounding differences only, rarely more than 1 ulp
-            for a, b in ((H[e, :n], H_ref[e, :n]), (ye[e, :n], ye_ref[e, :n])):
-                if a.numel():
-                    far = (a.double() - b.double()).abs() > 2.0 ** -7 * b.double().abs() + 1e-3
-                    assert float(far.double().mean()) < 1e-3
+            far.add(H[e, :n], H_ref[e, :n])
+            far.add(ye[e, :n], ye_ref[e, :n])
         else:
             assert_close(H[e, :n], H_ref[e, :n], atol=1e-5, rtol=1e-5, what=f"H[{e}]")
             assert_close(ye[e, :n], ye_ref[e, :n], atol=1e-5, rtol=1e-5, what=f"ye[{e}]")
         # rows past kept_cnt are never written
         assert bool(torch.isnan(H[e, n:].float()).all()) and bool(torch.isnan(ye[e, n:].float()).all())
+    # beyond the stated tolerance: rounding differences only, rarely more than 1 ulp
+    far.check(1e-3)
 
 
 @pytest.mark.parametrize("shape", sorted(FFN_SHAPES))
@@ -275,20 +299,19 @@ def test_expert_ffn_geglu(moe, cuda_device, shape):
     ye_ref, H_ref = oracle.expert_ffn(xe, W1, W2, kept, with_H=True, nthreads=threads(),
                                       kind="geglu")
     H, ye = H.cpu(), ye.cpu()
+    far = FarCount()
     for e in range(E):
         n = int(kept[e])
         assert_close(H[e, :n], H_ref[e, :n], what=f"H[{e}]")
         assert_close(ye[e, :n], ye_ref[e, :n], what=f"ye[{e}]")
-        # beyond the stated tolerance, rarely more than 1 ulp.  GEGLU's H is the product
-        # of two d-term sums, so the fp32 sums' rounding flips the bf16 rounding of H
-        # more often as d grows; each flip moves ye[t, :] by ulp(H) |W2|, which passes
-        # 1e-3 on the small |ye|.  At d = 2048 about 0.11 % of ye sits beyond, hence 2e-3.
-        far_max = 1e-3 if d < 2048 else 2e-3
-        for a, b in ((H[e, :n], H_ref[e, :n]), (ye[e, :n], ye_ref[e, :n])):
-            if a.numel():
-                far = (a.double() - b.double()).abs() > 2.0 ** -7 * b.double().abs() + 1e-3
-                assert float(far.double().mean()) < far_max
+        far.add(H[e, :n], H_ref[e, :n])
+        far.add(ye[e, :n], ye_ref[e, :n])
         assert bool(torch.isnan(H[e, n:].float()).all()) and bool(torch.isnan(ye[e, n:].float()).all())
+    # beyond the stated tolerance, rarely more than 1 ulp.  GEGLU's H is the product
+    # of two d-term sums, so the fp32 sums' rounding flips the bf16 rounding of H
+    # more often as d grows; each flip moves ye[t, :] by ulp(H) |W2|, which passes
+    # 1e-3 on the small |ye|.  At d = 2048 about 0.11 % of ye sits beyond, hence 2e-3.
+    far.check(1e-3 if d < 2048 else 2e-3)
 
 
 # ---------------------------------------------------------------------------
