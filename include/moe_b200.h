@@ -275,7 +275,10 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* expert
  * to y (ye is left untouched).
  * stage_events (nullable; a profiling hook): host array of 6 cudaEvent_t
  * (entries may be null) recorded on `stream` before the router and after
- * the router, the assignment, the dispatch, the expert FFN and the combine. */
+ * the router, the assignment, the dispatch, the expert FFN and the combine.
+ * The call only enqueues work on `stream` (no host synchronisation, no
+ * allocation), so it may be captured into a CUDA graph; the graph then
+ * reads and writes the same buffers on every replay. */
 int32_t moe_layer_forward(const moe_config* cfg, const void* x, const void* Wr, const float* bias,
                           const int32_t* domain_id, const void* W1, const void* W2, void* y,
                           void* workspace, size_t workspace_bytes, int32_t* status,
