@@ -79,7 +79,8 @@ class ClockSampler:
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+             "power.limit")
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
@@ -111,22 +112,38 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
+        return summarize_clock_lines(self.lines)
+
+
+def summarize_clock_lines(lines):
+    """Median SM clock and board power, the max clock and power limit, and every
+    throttle reason seen active, from ClockSampler.QUERY lines."""
+    sm, pw, mx, lim, reasons = [], [], None, None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx = float(parts[2])
+        except ValueError:
+            continue
+        try:
+            pw.append(float(parts[3]))
+        except ValueError:
+            pass
+        if len(parts) > 9:
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                lim = float(parts[9])
             except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                pass
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+            "reasons": sorted(reasons), "samples": len(sm),
+            "power_w": statistics.median(pw) if pw else None, "power_limit_w": lim}
 
 
 def dist_setup(args):

@@ -58,3 +58,21 @@ def test_stage_roofline_picks_the_slower_roof():
     r = bench.stage_roofline({"a": (1e9, 0.5e12), "b": (2e9, 0.0)}, {"a": 1000.0, "b": 4.0}, peaks)
     assert r["a"]["bound"] == "tensor" and r["a"]["frac"] == 0.5
     assert r["b"]["bound"] == "hbm" and r["b"]["frac"] == 0.5 and r["b"]["gbs"] == 500.0
+
+
+def test_clock_summary_lines():
+    """nvidia-smi lines in ClockSampler.QUERY order: medians of SM clock and board
+    power, the last max clock and power limit, every throttle reason seen active;
+    an unreadable power field is skipped, a short line ignored."""
+    lines = [
+        "0, 1200, 1965, 998.50, 0x4, Not Active, Not Active, Not Active, Active, 1000.00",
+        "0, 1300, 1965, 1001.20, 0x4, Not Active, Not Active, Not Active, Active, 1000.00",
+        "0, 1250, 1965, [N/A], 0x0, Not Active, Not Active, Active, Not Active, 1000.00",
+        "0, 1250",
+    ]
+    s = bench.summarize_clock_lines(lines)
+    assert s["sm_mhz"] == 1250.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["power_w"] == pytest.approx((998.5 + 1001.2) / 2)
+    assert s["power_limit_w"] == 1000.0
+    assert s["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    assert bench.summarize_clock_lines([])["sm_mhz"] is None
