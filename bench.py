@@ -37,8 +37,10 @@ L2_BYTES = 126 * 1024 * 1024
 # capture of the kernels as shipped (the profile named beside each number).
 # A workload without a capture of its current kernels reports null.
 FFN_TRAFFIC = {
-    "switch_base": (1240.836e6 + 29.177e6, "profiles/ffn_tc_switch_base.md"),
-    "xmoe_top2": (604.122e6 + 228.916e6 + 825.805e6 + 55.799e6, "profiles/gemm_pair_xmoe_top2.md"),
+    "switch_base": (1242.470e6 + 28.536e6, "profiles/ffn_tc_switch_base.md"),
+    "xmoe_top2": (604.202e6 + 228.670e6 + 825.849e6 + 56.016e6, "profiles/gemm_pair_xmoe_top2.md"),
+    "skewed_switch": (2218.970e6 + 73.474e6 + 2434.246e6 + 17.644e6,
+                      "profiles/gemm_tc_ffn_skewed_switch.md"),
     # captured on 8 experts (same capacity and per-expert load), scaled by 64 / 8
     "pangu_rre": ((1194.575e6 + 103.069e6) * 8, "profiles/ffn_pair_pangu_rre.md"),
 }
