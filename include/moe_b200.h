@@ -84,7 +84,7 @@ enum moe_status_bits {
 
 /* One MoE layer.  56 bytes, no padding. */
 typedef struct moe_config {
-  int64_t T;          /* tokens in the batch (>= 0)                                    */
+  int64_t T;          /* tokens in the batch (>= 0; T * k <= 2^31 - 1)                 */
   int32_t d_model;    /* token width d                                                 */
   int32_t d_ff;       /* expert hidden width f                                         */
   int32_t E;          /* experts, 1..256                                               */

@@ -82,6 +82,8 @@ int32_t check_cfg(const moe_config* c) {
   const int64_t EC = int64_t(c->E) * c->capacity;
   if (EC > kI32Max || int64_t(c->E) * c->d_ff * 2 > kI32Max || int64_t(c->E) * c->d_model > kI32Max)
     return fail(MOE_ERR_UNSUPPORTED, "E*C, E*d_ff or E*d_model exceeds 2^31-1 rows");
+  // per-expert arrival counts, slots and the choice index are 32-bit
+  if (c->T * c->k > kI32Max) return fail(MOE_ERR_UNSUPPORTED, "T*k exceeds 2^31-1 choices");
   return MOE_OK;
 }
 

@@ -65,6 +65,7 @@ def cfg(moe, **kw):
     (dict(capacity_=-1), -1), (dict(d_model=100), -2), (dict(d_ff=96), -2),
     (dict(mode="rre", k=2, num_groups=8), -1), (dict(mode="rre", num_groups=3), -1),
     (dict(T=-5), -1), (dict(expert="geglu", dtype="f32"), -2),
+    (dict(T=2 ** 30, k=2), -2),  # T * k = 2^31 choices: counts and slots are 32-bit
 ])
 def test_config_rejections(moe, kw, code):
     c = cfg(moe, **kw)
@@ -221,6 +222,8 @@ def _expected_check(T, d, f, E, k, C, mode, G, dtype, expert):
     if (dtype == 0 and (d % 64 or f % 64)) or (dtype == 1 and (d % 4 or f % 4)):
         return -2
     if E * C > I32 or E * f * 2 > I32 or E * d > I32:
+        return -2
+    if T * k > I32:
         return -2
     return 0
 
