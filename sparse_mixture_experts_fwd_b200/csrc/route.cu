@@ -469,6 +469,13 @@ int32_t launch_assign(const moe_config& c, const int32_t* expert_idx, int32_t* s
   p.arrivals = arrivals;
   p.kept_cnt = kept_cnt;
   p.n_dropped = n_dropped;
+  // on every launch: a function attribute belongs to the current context, the
+  // cached cluster size to the device
+  if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(assign_smem_bytes(256))) != cudaSuccess ||
+      cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+    return check_launch("cudaFuncSetAttribute(assign_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(nb));
   cfg.blockDim = dim3(kAssignThreads);

@@ -445,6 +445,11 @@ int32_t launch_router_pair(const moe_config& c, const void* x, const void* Wr, R
                  static_cast<uint32_t>(C::kBRows));
   if (rc != MOE_OK) return rc;
   auto kern = router_topk_pair_kernel<BN>;
+  // on every launch: a function attribute belongs to the current context, the
+  // cached pair count to the device
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return check_launch("cudaFuncSetAttribute(router_topk_pair_kernel)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<int64_t>(pairs, p.tiles)));
   cfg.blockDim = dim3(kThreads);
