@@ -76,3 +76,33 @@ def test_clock_summary_lines():
     assert s["power_limit_w"] == 1000.0
     assert s["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
     assert bench.summarize_clock_lines([])["sm_mhz"] is None
+
+
+def test_reference_arm_json_line():
+    """`bench.py --impl reference` (the CPU oracle, no GPU) prints one JSON line
+    with the contract's keys: the oracle's rate as value, cpu_baseline and an
+    e2e object with no host-device bytes."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", "switch_base", "--steps", "1", "--warmup", "1",
+                          "--cpu-seconds", "1"],
+                         capture_output=True, text=True, timeout=600, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] == 1
+    assert d["config"]["workload"] == "switch_base"
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
